@@ -1,0 +1,300 @@
+// Dispatch table: rows keyed (op, padded M, N, K) naming a kernel configuration,
+// the padded-M lookup walk, and the lookup census.
+//
+// Walk ([aiter#7752] "[Perf] Retune gfx942 Qwen3.8-27B a8w8 blockscale decode rows
+// for cold weights", section "PR-specific question"): probe exact M; then the next
+// power of two if M < 16, or the next multiple of 16 if 16 <= M <= 256; then the next
+// power of two; else miss. [cookbook#8] "Two amplifiers": M = 6016 therefore runs the
+// row tuned for 8192. A miss runs the per-shape default configuration
+// ([mi210 docs/43] section 6: a miss returns None and the default kernel runs).
+// Census ([cookbook#8], coverage_report.py review): lookups are counted per distinct
+// key so duplicates collapse.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "internal.h"
+
+namespace fp8bs {
+
+// ------------------------------------------------------------ configurations
+static const KernelConfig kConfigs[] = {
+    // name                    op                          path       bn  sk  depth
+    {"a8w8_gemv_d2", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemv, 0, 1, 2},
+    {"a8w8_gemv_d3", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemv, 0, 1, 3},
+    {"a8w8_gemv_d4", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemv, 0, 1, 4},
+    {"a8w8_tc_bn128", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 128, 1, 0},
+    {"a8w8_tc_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 256, 1, 0},
+    {"bf16_gemv_d2", FP8BS_OP_BF16, kPathGemv, 0, 1, 2},
+    {"bf16_gemv_d4", FP8BS_OP_BF16, kPathGemv, 0, 1, 4},
+    {"bf16_tc_bn32", FP8BS_OP_BF16, kPathTc, 32, 1, 0},
+    {"bf16_tc_bn64", FP8BS_OP_BF16, kPathTc, 64, 1, 0},
+    {"bf16_tc_bn128", FP8BS_OP_BF16, kPathTc, 128, 1, 0},
+    {"bf16_tc_bn192", FP8BS_OP_BF16, kPathTc, 192, 1, 0},
+    {"bf16_tc_bn256", FP8BS_OP_BF16, kPathTc, 256, 1, 0},
+};
+static constexpr int kNumConfigs = sizeof(kConfigs) / sizeof(kConfigs[0]);
+
+const KernelConfig* find_config(int op, const char* name) {
+  if (!name) return nullptr;
+  for (const auto& c : kConfigs)
+    if (c.op == op && std::strcmp(c.name, name) == 0) return &c;
+  return nullptr;
+}
+
+const KernelConfig* const* list_configs(int op, int* count) {
+  static const KernelConfig* lists[FP8BS_NUM_OPS][kNumConfigs];
+  static int counts[FP8BS_NUM_OPS];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    for (const auto& c : kConfigs) lists[c.op][counts[c.op]++] = &c;
+  });
+  *count = counts[op];
+  return lists[op];
+}
+
+const KernelConfig* default_config(int op, int64_t M, int64_t N, int64_t K) {
+  (void)K;
+  if (op == FP8BS_OP_A8W8_BLOCKSCALE) {
+    if (M <= kGemvMaxM) return find_config(op, M <= 8 ? "a8w8_gemv_d4" : M <= 16 ? "a8w8_gemv_d3" : "a8w8_gemv_d2");
+    if (N % 256 == 0) return find_config(op, "a8w8_tc_bn256");
+    return find_config(op, "a8w8_tc_bn128");
+  }
+  if (M <= kGemvMaxM) return find_config(op, M <= 16 ? "bf16_gemv_d4" : "bf16_gemv_d2");
+  if (N <= 256 && (N == 32 || N == 64 || N == 128 || N == 192 || N == 256)) {
+    char nm[32];
+    std::snprintf(nm, sizeof nm, "bf16_tc_bn%d", int(N));
+    return find_config(op, nm);
+  }
+  if (N % 256 == 0) return find_config(op, "bf16_tc_bn256");
+  if (N % 192 == 0) return find_config(op, "bf16_tc_bn192");
+  if (N % 128 == 0) return find_config(op, "bf16_tc_bn128");
+  if (N % 64 == 0) return find_config(op, "bf16_tc_bn64");
+  return find_config(op, "bf16_tc_bn32");
+}
+
+// ------------------------------------------------------------ table + census
+namespace {
+
+using Key = std::tuple<int, int64_t, int64_t, int64_t>;                        // op, M, N, K
+using CensusKey = std::tuple<int, int64_t, int64_t, int64_t, int64_t, std::string>;  // op, M, N, K, padded_M, cfg
+
+struct State {
+  std::mutex mu;
+  std::map<Key, const KernelConfig*> rows;
+  std::map<CensusKey, uint64_t> census;
+  uint64_t hits[FP8BS_NUM_OPS] = {0, 0};
+  uint64_t misses[FP8BS_NUM_OPS] = {0, 0};
+  bool log = false;
+};
+
+void add_builtin_rows(std::map<Key, const KernelConfig*>& rows) {
+  // Rows for the decode / prefill projections at the tuner's M ladder: powers of two,
+  // multiples of 16 up to 256. The configuration named is the measured choice for
+  // the shape where one has been made, else the default heuristic.
+  const int64_t nk[][2] = {{5120, 6144}, {14336, 5120}, {16384, 5120}, {34816, 5120}};
+  std::vector<int64_t> ms = {1, 2, 4, 8};
+  for (int64_t m = 16; m <= 256; m += 16) ms.push_back(m);
+  for (int64_t m = 512; m <= 8192; m *= 2) ms.push_back(m);
+  for (const auto& p : nk)
+    for (int64_t m : ms)
+      rows[Key{FP8BS_OP_A8W8_BLOCKSCALE, m, p[0], p[1]}] = default_config(FP8BS_OP_A8W8_BLOCKSCALE, m, p[0], p[1]);
+  const int64_t bnk[][2] = {{256, 6144}, {32, 6144}, {384, 5120}, {1024, 5120}, {128, 512}};
+  const int64_t bms[] = {1, 32, 576, 4096, 16384};
+  for (const auto& p : bnk)
+    for (int64_t m : bms) rows[Key{FP8BS_OP_BF16, m, p[0], p[1]}] = default_config(FP8BS_OP_BF16, m, p[0], p[1]);
+}
+
+State& state() {
+  static State* s = [] {
+    auto* st = new State();
+    add_builtin_rows(st->rows);
+    const char* e = std::getenv("FP8BS_LOG_DISPATCH");
+    st->log = e && e[0] == '1';
+    return st;
+  }();
+  return *s;
+}
+
+int64_t next_pow2(int64_t m) {
+  int64_t p = 1;
+  while (p < m) p <<= 1;
+  return p;
+}
+
+}  // namespace
+
+const KernelConfig* dispatch(int op, int64_t M, int64_t N, int64_t K, bool record, int64_t* padded_M, bool* hit) {
+  State& st = state();
+  int64_t probes[3];
+  int np = 0;
+  probes[np++] = M;
+  if (M < 16)
+    probes[np++] = next_pow2(M);
+  else if (M <= 256)
+    probes[np++] = (M + 15) / 16 * 16;
+  probes[np++] = next_pow2(M);
+
+  std::lock_guard<std::mutex> lk(st.mu);
+  const KernelConfig* cfg = nullptr;
+  int64_t pm = 0;
+  for (int i = 0; i < np && !cfg; ++i) {
+    auto it = st.rows.find(Key{op, probes[i], N, K});
+    if (it != st.rows.end()) {
+      cfg = it->second;
+      pm = probes[i];
+    }
+  }
+  const bool is_hit = cfg != nullptr;
+  if (!cfg) cfg = default_config(op, M, N, K);
+  if (padded_M) *padded_M = pm;
+  if (hit) *hit = is_hit;
+  if (record && cfg) {
+    (is_hit ? st.hits : st.misses)[op]++;
+    auto& cnt = st.census[CensusKey{op, M, N, K, pm, cfg->name}];
+    if (cnt++ == 0 && st.log)
+      std::fprintf(stderr, "[fp8bs] lookup op=%d M=%lld N=%lld K=%lld padded_M=%lld %s cfg=%s\n", op,
+                   (long long)M, (long long)N, (long long)K, (long long)pm, is_hit ? "hit" : "miss", cfg->name);
+  }
+  return cfg;
+}
+
+}  // namespace fp8bs
+
+using namespace fp8bs;
+
+extern "C" {
+
+__attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_lookup(int op, int64_t M, int64_t N, int64_t K,
+                                                                          int record, int64_t* padded_M, int* hit,
+                                                                          char* cfg, size_t cfg_len) {
+  if (op < 0 || op >= FP8BS_NUM_OPS || M <= 0 || N <= 0 || K <= 0) return FP8BS_ERR_INVALID_ARG;
+  bool h = false;
+  int64_t pm = 0;
+  const KernelConfig* c = dispatch(op, M, N, K, record != 0, &pm, &h);
+  if (!c) return FP8BS_ERR_UNSUPPORTED;
+  if (padded_M) *padded_M = pm;
+  if (hit) *hit = h ? 1 : 0;
+  if (cfg && cfg_len) {
+    std::strncpy(cfg, c->name, cfg_len - 1);
+    cfg[cfg_len - 1] = 0;
+  }
+  return FP8BS_OK;
+}
+
+__attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_set_row(int op, int64_t M, int64_t N, int64_t K,
+                                                                           const char* cfg) {
+  if (op < 0 || op >= FP8BS_NUM_OPS || M <= 0 || N <= 0 || K <= 0 || !cfg) return FP8BS_ERR_INVALID_ARG;
+  const KernelConfig* c = find_config(op, cfg);
+  if (!c) return FP8BS_ERR_INVALID_ARG;
+  if (c->path == kPathGemv && M > kGemvMaxM) return FP8BS_ERR_UNSUPPORTED;
+  State& st = state();
+  std::lock_guard<std::mutex> lk(st.mu);
+  st.rows[Key{op, M, N, K}] = c;
+  return FP8BS_OK;
+}
+
+__attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_reset_table(int keep_builtin) {
+  State& st = state();
+  std::lock_guard<std::mutex> lk(st.mu);
+  st.rows.clear();
+  if (keep_builtin) add_builtin_rows(st.rows);
+  return FP8BS_OK;
+}
+
+__attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_list_configs(int op, char* buf, size_t len) {
+  if (op < 0 || op >= FP8BS_NUM_OPS || !buf || !len) return FP8BS_ERR_INVALID_ARG;
+  int n = 0;
+  const KernelConfig* const* l = list_configs(op, &n);
+  std::string s;
+  for (int i = 0; i < n; ++i) {
+    s += l[i]->name;
+    s += '\n';
+  }
+  std::strncpy(buf, s.c_str(), len - 1);
+  buf[len - 1] = 0;
+  return s.size() < len ? FP8BS_OK : FP8BS_ERR_INVALID_ARG;
+}
+
+__attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_stats(int op, uint64_t* hits, uint64_t* misses,
+                                                                         uint64_t* distinct_hits,
+                                                                         uint64_t* distinct_misses) {
+  if (op < 0 || op >= FP8BS_NUM_OPS) return FP8BS_ERR_INVALID_ARG;
+  State& st = state();
+  std::lock_guard<std::mutex> lk(st.mu);
+  uint64_t dh = 0, dm = 0;
+  for (const auto& kv : st.census) {
+    if (std::get<0>(kv.first) != op) continue;
+    (std::get<4>(kv.first) != 0 ? dh : dm)++;
+  }
+  if (hits) *hits = st.hits[op];
+  if (misses) *misses = st.misses[op];
+  if (distinct_hits) *distinct_hits = dh;
+  if (distinct_misses) *distinct_misses = dm;
+  return FP8BS_OK;
+}
+
+__attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_reset_stats(void) {
+  State& st = state();
+  std::lock_guard<std::mutex> lk(st.mu);
+  st.census.clear();
+  for (int i = 0; i < FP8BS_NUM_OPS; ++i) st.hits[i] = st.misses[i] = 0;
+  return FP8BS_OK;
+}
+
+__attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_dump_json(char* buf, size_t len) {
+  if (!buf || !len) return FP8BS_ERR_INVALID_ARG;
+  State& st = state();
+  std::string s = "[";
+  {
+    std::lock_guard<std::mutex> lk(st.mu);
+    bool first = true;
+    char line[256];
+    for (const auto& kv : st.census) {
+      const auto& k = kv.first;
+      std::snprintf(line, sizeof line,
+                    "%s{\"op\":%d,\"M\":%lld,\"N\":%lld,\"K\":%lld,\"padded_M\":%lld,\"hit\":%s,\"cfg\":\"%s\","
+                    "\"count\":%llu}",
+                    first ? "" : ",", std::get<0>(k), (long long)std::get<1>(k), (long long)std::get<2>(k),
+                    (long long)std::get<3>(k), (long long)std::get<4>(k), std::get<4>(k) ? "true" : "false",
+                    std::get<5>(k).c_str(), (unsigned long long)kv.second);
+      s += line;
+      first = false;
+    }
+  }
+  s += "]";
+  if (s.size() >= len) {
+    buf[0] = 0;
+    return FP8BS_ERR_INVALID_ARG;
+  }
+  std::memcpy(buf, s.c_str(), s.size() + 1);
+  return FP8BS_OK;
+}
+
+__attribute__((visibility("default"))) uint64_t fp8bs_dispatch_table_hash(void) {
+  State& st = state();
+  std::lock_guard<std::mutex> lk(st.mu);
+  uint64_t h = 1469598103934665603ull;
+  auto mix = [&h](const void* p, size_t n) {
+    const unsigned char* b = static_cast<const unsigned char*>(p);
+    for (size_t i = 0; i < n; ++i) {
+      h ^= b[i];
+      h *= 1099511628211ull;
+    }
+  };
+  for (const auto& kv : st.rows) {
+    int op = std::get<0>(kv.first);
+    int64_t v[3] = {std::get<1>(kv.first), std::get<2>(kv.first), std::get<3>(kv.first)};
+    mix(&op, sizeof op);
+    mix(v, sizeof v);
+    mix(kv.second->name, std::strlen(kv.second->name));
+  }
+  return h;
+}
+
+}  // extern "C"

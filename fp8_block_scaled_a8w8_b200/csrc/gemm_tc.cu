@@ -1,0 +1,439 @@
+// Tensor-core GEMM for prefill-sized M: tcgen05.mma with TMEM accumulators, operands
+// staged in shared memory by TMA (128-byte swizzle), persistent and warp-specialised.
+//
+//   warp 0        TMA producer: one 128-row A box and one BN-row W box per K block
+//   warp 1        TMEM allocator and MMA issuer (one elected thread)
+//   warps 2..9    epilogue: TMEM -> registers -> bf16/f32 -> global
+//
+// a8w8 block scale: a 128-wide K group is one K block. Each group's four
+// tcgen05.mma (K = 32 each) write a fresh float32 partial P_g into one of two TMEM
+// buffers; while the tensor core fills the other buffer with group g+1, the epilogue
+// warps read P_g and add a_scale[row,g] * w_scale[col/128,g] * P_g into float32
+// register accumulators -- the block-scale definition, group by group
+// ([cookbook#8]: 128x128 weight blocks; 1x128 activation groups), with the
+// scale promotion overlapped with the next group's MMAs.
+// bf16: the K blocks (64 columns) accumulate in TMEM; the two buffers alternate
+// between output tiles so the epilogue of one tile overlaps the next tile's MMAs.
+//
+// Every wait is bounded (kWaitLimitNs); a timed-out wait raises the CTA's abort flag
+// and the device status word, the roles leave their loops, in-flight TMA loads and
+// MMAs are drained (bounded) and TMEM is freed before the CTA exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fp8bs {
+
+// Status word of the kernels in this file (bit kStatusTimeout: a bounded wait gave up).
+static __device__ unsigned int g_tc_status = 0;
+
+unsigned int take_device_status() {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_tc_status, sizeof v) != cudaSuccess) return ~0u;
+  if (v) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_tc_status, &zero, sizeof zero) != cudaSuccess) return ~0u;
+  }
+  return v;
+}
+
+constexpr int kTcThreads = 320;
+constexpr int kBM = 128;
+constexpr int kKBlockBytes = 128;
+
+template <bool kFp8, int BN>
+struct TcCfg {
+  static constexpr int kABytes = kBM * kKBlockBytes;
+  static constexpr int kBBytes = BN * kKBlockBytes;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+  static constexpr int kTmemCols = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128 : (2 * BN <= 256) ? 256 : 512;
+  static constexpr int kHalfCols = BN / 2;  // columns per epilogue warp
+  static constexpr int kChunk = kHalfCols >= 32 ? 32 : kHalfCols;
+  static constexpr int kChunks = kHalfCols / kChunk;
+  static constexpr uint32_t kIdesc = make_idesc(kFp8 ? kFmtE4M3 : kFmtBF16, kFp8 ? kFmtE4M3 : kFmtBF16, kBM, BN);
+  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(kHalfCols % kChunk == 0, "chunking");
+  static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "N tile");
+};
+
+struct TcParams {
+  const float* a_scale;  // [M, G] (a8w8)
+  const float* w_scale;  // [ceil(N/128), G] (a8w8)
+  void* out;             // [M, N]
+  int M, N, K;
+  int kblocks;           // K blocks of 128 bytes
+  int m_tiles, n_tiles;
+  int out_fp32;
+};
+
+__device__ __forceinline__ void tmem_ld_chunk16(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+template <int kChunk>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[32]) {
+  if constexpr (kChunk == 32)
+    tmem_ld_32x32b_x32(taddr, r);
+  else
+    tmem_ld_chunk16(taddr, r);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Store kChunk consecutive columns of one row (bf16 or f32), masked at N.
+template <int kChunk>
+__device__ __forceinline__ void store_row_chunk(const TcParams& p, int row, int col, const float* v) {
+  if (row >= p.M) return;
+  if (p.out_fp32) {
+    float* dst = static_cast<float*>(p.out) + int64_t(row) * p.N + col;
+#pragma unroll
+    for (int j = 0; j < kChunk; j += 4)
+      if (col + j < p.N) *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+  } else {
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) + int64_t(row) * p.N + col;
+#pragma unroll
+    for (int j = 0; j < kChunk; j += 8)
+      if (col + j < p.N)
+        *reinterpret_cast<uint4*>(dst + j) =
+            make_uint4(pack_bf16x2(v[j], v[j + 1]), pack_bf16x2(v[j + 2], v[j + 3]), pack_bf16x2(v[j + 4], v[j + 5]),
+                       pack_bf16x2(v[j + 6], v[j + 7]));
+  }
+}
+
+template <bool kFp8, int BN>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+  using C = TcCfg<kFp8, BN>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* tiles = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(S) * C::kStageBytes);
+  // bars: full[S], empty[S], tmem_full[2], tmem_empty[2], drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + S + s); };
+  auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * S + b); };
+  auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * S + 2 + b); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * S + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 8);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int tiles_total = p.m_tiles * p.n_tiles;
+  const int KB = p.kblocks;
+  const int G = p.K / 128;  // scale groups (a8w8)
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      int last_it[8];
+      for (int s = 0; s < S; ++s) last_it[s] = -1;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles_total && ok; tile += gridDim.x) {
+        const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait_bounded(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, &g_tc_status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = smem_u32(tiles + size_t(s) * C::kStageBytes);
+          const uint32_t b_dst = a_dst + C::kABytes;
+          mbar_arrive_expect_tx(full_bar(s), C::kStageBytes);
+          const int kx = kFp8 ? kb * 128 : kb * 64;
+          tma_load_2d(a_dst, &tmA, full_bar(s), kx, tm * kBM);
+          tma_load_2d(b_dst, &tmB, full_bar(s), kx, tn * BN);
+          last_it[s] = it;
+        }
+      }
+      // drain: wait (bounded, regardless of abort) for every issued load to land
+      for (int s = 0; s < S; ++s) {
+        if (last_it[s] < 0) continue;
+        const uint32_t par = (last_it[s] / S) & 1;
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(full_bar(s), par))
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_tc_status, kStatusTimeout);
+            break;
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, acc_it = 0, tile_it = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int tile = blockIdx.x; tile < tiles_total && ok; tile += gridDim.x, ++tile_it) {
+        uint32_t d_tmem = 0;
+        int tb = tile_it & 1;
+        if (!kFp8) {
+          if (!mbar_wait_bounded(tempty_bar(tb), ((tile_it >> 1) & 1) ^ 1, abort_flag, &g_tc_status)) break;
+          tc_fence_after();
+          d_tmem = tmem_base + uint32_t(tb * BN);
+        }
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait_bounded(full_bar(s), (it / S) & 1, abort_flag, &g_tc_status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          int b = 0;
+          if (kFp8) {
+            b = acc_it & 1;
+            if (!mbar_wait_bounded(tempty_bar(b), ((acc_it >> 1) & 1) ^ 1, abort_flag, &g_tc_status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            d_tmem = tmem_base + uint32_t(b * BN);
+          }
+          const uint32_t a_addr = smem_u32(tiles + size_t(s) * C::kStageBytes);
+          const uint64_t adesc = sw128_kmajor_desc(a_addr);
+          const uint64_t bdesc = sw128_kmajor_desc(a_addr + C::kABytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t acc = kFp8 ? (kk > 0) : (kb > 0 || kk > 0);
+            if (kFp8)
+              umma_f8f6f4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, C::kIdesc, acc);
+            else
+              umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, C::kIdesc, acc);
+          }
+          issued = true;
+          umma_commit(empty_bar(s));
+          if (kFp8) {
+            umma_commit(tfull_bar(b));
+            ++acc_it;
+          }
+        }
+        if (!kFp8 && ok) umma_commit(tfull_bar(tb));
+      }
+      // drain: every MMA issued by this thread has completed once drain_bar flips
+      if (issued) {
+        umma_commit(drain_bar);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain_bar, 0))
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_tc_status, kStatusTimeout);
+            break;
+          }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue warps 2..9
+    const int q = warp & 3;          // TMEM lane quarter this warp may access
+    const int h = (warp - 2) >> 2;   // column half
+    const int row_in_tile = 32 * q + lane;
+    const uint32_t lane_addr = tmem_base + (uint32_t(32 * q) << 16);
+    int acc_it = 0, tile_it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles_total && ok; tile += gridDim.x, ++tile_it) {
+      const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
+      const int row = tm * kBM + row_in_tile;
+      const int col0 = tn * BN + h * C::kHalfCols;
+      if constexpr (kFp8) {
+        float acc[C::kHalfCols];
+#pragma unroll
+        for (int j = 0; j < C::kHalfCols; ++j) acc[j] = 0.f;
+        const int nbw = col0 >> 7;  // W scale block of this warp's columns
+        const bool nb_ok = col0 < p.N;
+        const float* asrow = p.a_scale + int64_t(row < p.M ? row : 0) * G;
+        const bool row_ok = row < p.M;
+        float sa0 = row_ok ? __ldg(asrow + 0) : 0.f;
+        float sa1 = (row_ok && KB > 1) ? __ldg(asrow + 1) : 0.f;
+        for (int kb = 0; kb < KB; ++kb) {
+          const float sa = sa0;
+          sa0 = sa1;
+          sa1 = (row_ok && kb + 2 < KB) ? __ldg(asrow + kb + 2) : 0.f;
+          const float sw = nb_ok ? __ldg(p.w_scale + int64_t(nbw) * G + kb) : 0.f;
+          const float sc = sa * sw;
+          const int b = acc_it & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (acc_it >> 1) & 1, abort_flag, &g_tc_status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t t_addr = lane_addr + uint32_t(b * BN + h * C::kHalfCols);
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c) {
+            uint32_t r[32];
+            tmem_ld<C::kChunk>(t_addr + c * C::kChunk, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < C::kChunk; ++j) acc[c * C::kChunk + j] = fmaf(__uint_as_float(r[j]), sc, acc[c * C::kChunk + j]);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(b));
+          ++acc_it;
+        }
+        if (!ok) break;
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c) store_row_chunk<C::kChunk>(p, row, col0 + c * C::kChunk, acc + c * C::kChunk);
+      } else {
+        const int b = tile_it & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (tile_it >> 1) & 1, abort_flag, &g_tc_status)))
+          break;
+        tc_fence_after();
+        const uint32_t t_addr = lane_addr + uint32_t(b * BN + h * C::kHalfCols);
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c) {
+          uint32_t r[32];
+          tmem_ld<C::kChunk>(t_addr + c * C::kChunk, r);
+          tmem_ld_wait();
+          float v[C::kChunk];
+#pragma unroll
+          for (int j = 0; j < C::kChunk; ++j) v[j] = __uint_as_float(r[j]);
+          store_row_chunk<C::kChunk>(p, row, col0 + c * C::kChunk, v);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(b));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 2-D K-major tensor map: rows of `cols` elements, box = 128 bytes x box_rows, 128-byte swizzle.
+static bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const int esz = fp8 ? 1 : 2;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols * esz)};
+  cuuint32_t box[2] = {cuuint32_t(kKBlockBytes / esz), cuuint32_t(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  std::memset(m, 0, sizeof(*m));
+  CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool kFp8, int BN>
+static int launch_tc_t(const void* A, const void* W, const TcParams& prm, void* stream) {
+  using C = TcCfg<kFp8, BN>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_tc_kernel<kFp8, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(C::kSmemBytes));
+  });
+  if (attr_err != cudaSuccess) return int(attr_err);
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, A, kFp8, prm.M, prm.K, kBM) || !make_map(&mb, W, kFp8, prm.N, prm.K, BN))
+    return int(cudaErrorInvalidValue);
+  const int tiles = prm.m_tiles * prm.n_tiles;
+  const int grid = std::min(tiles, device_sm_count());
+  gemm_tc_kernel<kFp8, BN><<<grid, kTcThreads, C::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(ma, mb, prm);
+  return int(cudaGetLastError());
+}
+
+size_t tc_workspace_bytes(int, int64_t, int64_t, int64_t, const KernelConfig&) { return 0; }
+
+static TcParams make_params(const float* a_scale, const float* w_scale, void* out, int64_t M, int64_t N, int64_t K,
+                            int bn, bool fp8, int out_fp32) {
+  TcParams p{};
+  p.a_scale = a_scale;
+  p.w_scale = w_scale;
+  p.out = out;
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.kblocks = int(fp8 ? K / 128 : K / 64);
+  p.m_tiles = int((M + kBM - 1) / kBM);
+  p.n_tiles = int((N + bn - 1) / bn);
+  p.out_fp32 = out_fp32;
+  return p;
+}
+
+int launch_tc_a8w8(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W,
+                   const float* w_scale, void* out, int64_t M, int64_t N, int64_t K, void*, void* stream) {
+  const TcParams p = make_params(a_scale, w_scale, out, M, N, K, cfg.bn, true, 0);
+  switch (cfg.bn) {
+    case 128: return launch_tc_t<true, 128>(A, W, p, stream);
+    case 256: return launch_tc_t<true, 256>(A, W, p, stream);
+    default: return int(cudaErrorInvalidValue);
+  }
+}
+
+int launch_tc_bf16(const KernelConfig& cfg, const void* A, const void* W, void* out, int out_fp32, int64_t M,
+                   int64_t N, int64_t K, void*, void* stream) {
+  const TcParams p = make_params(nullptr, nullptr, out, M, N, K, cfg.bn, false, out_fp32);
+  switch (cfg.bn) {
+    case 32: return launch_tc_t<false, 32>(A, W, p, stream);
+    case 64: return launch_tc_t<false, 64>(A, W, p, stream);
+    case 128: return launch_tc_t<false, 128>(A, W, p, stream);
+    case 192: return launch_tc_t<false, 192>(A, W, p, stream);
+    case 256: return launch_tc_t<false, 256>(A, W, p, stream);
+    default: return int(cudaErrorInvalidValue);
+  }
+}
+
+}  // namespace fp8bs

@@ -1,0 +1,60 @@
+// Host-side internals shared by the C ABI (api.cu), the dispatch table
+// (dispatch.cpp) and the kernel launchers (*.cu).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "fp8bs.h"
+
+namespace fp8bs {
+
+enum Path : int {
+  kPathGemv = 0,  // weight-streaming split-K kernel (mma.sync, small M)
+  kPathTc = 1,    // tcgen05/TMEM tensor-core kernel fed by TMA
+};
+
+// One kernel configuration a dispatch-table row can name.
+struct KernelConfig {
+  const char* name;
+  int op;           // FP8BS_OP_*
+  int path;         // Path
+  int bn;           // tensor-core path: N tile (columns of W per CTA)
+  int split_k;      // tensor-core path: K splits (1 = none)
+  int gemv_depth;   // weight-streaming path: units in flight per warp
+};
+
+// Registry of every configuration (static storage).
+const KernelConfig* find_config(int op, const char* name);
+const KernelConfig* const* list_configs(int op, int* count);
+// Heuristic configuration for a shape with no table row.
+const KernelConfig* default_config(int op, int64_t M, int64_t N, int64_t K);
+// Table lookup with the padded-M walk; record != 0 counts it in the census.
+const KernelConfig* dispatch(int op, int64_t M, int64_t N, int64_t K, bool record, int64_t* padded_M, bool* hit);
+
+// Largest M the weight-streaming path handles (8 tokens per mma.sync N block, 4 blocks).
+constexpr int64_t kGemvMaxM = 32;
+
+// Reads and clears the device-side status word (~0u on a CUDA error).
+unsigned int take_device_status();
+
+// Device properties, cached per device.
+int device_sm_count();
+
+// ---- launchers (return a cudaError_t value as int; 0 = success) ----
+int launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q, float* scale, void* stream);
+int launch_quant_weight(const float* w, int64_t N, int64_t K, void* q, float* scale, void* stream);
+
+size_t gemv_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, const KernelConfig& cfg);
+int launch_gemv_a8w8(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W,
+                     const float* w_scale, void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream);
+int launch_gemv_bf16(const KernelConfig& cfg, const void* A, const void* W, void* out, int out_fp32, int64_t M,
+                     int64_t N, int64_t K, void* ws, void* stream);
+
+size_t tc_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, const KernelConfig& cfg);
+int launch_tc_a8w8(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W,
+                   const float* w_scale, void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream);
+int launch_tc_bf16(const KernelConfig& cfg, const void* A, const void* W, void* out, int out_fp32, int64_t M,
+                   int64_t N, int64_t K, void* ws, void* stream);
+
+}  // namespace fp8bs

@@ -1,0 +1,117 @@
+// Activation (per token, 1x128 group) and weight (128x128 block) quantisers.
+//
+// scale = amax / 448 and code = e4m3_rn_satfinite(x / scale), both divisions IEEE
+// float32 round-to-nearest (__fdiv_rn), the conversion the hardware
+// cvt.rn.satfinite.e4m3x2.f32 -- so the codes and scales equal the CPU
+// oracle's bit for bit. A group whose amax is 0 gets scale 0 and codes +-0.
+// ([cookbook#8]: the checkpoint is block quantised, weight_block_size [128,128].)
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fp8bs {
+
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ float quant_div(float x, float s) { return s == 0.f ? x : __fdiv_rn(x, s); }
+
+__device__ __forceinline__ uint32_t cvt4_e4m3(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return (lo & 0xFFFFu) | (hi << 16);
+}
+
+// One half-warp per group: 16 lanes x 8 bf16 = 128 values; a warp takes two groups.
+__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
+                                                        int64_t ld_x, uint8_t* __restrict__ q,
+                                                        float* __restrict__ scale) {
+  const int64_t G = K / 128;
+  const int64_t total = M * G;
+  const int lane = threadIdx.x & 31;
+  const int half = lane >> 4;
+  const int hl = lane & 15;
+  const int64_t warp = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t gp = warp * 2; gp < total; gp += nwarps * 2) {
+    const int64_t gi = gp + half;
+    const bool valid = gi < total;
+    const int64_t m = valid ? gi / G : 0;
+    const int64_t g = valid ? gi - m * G : 0;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (valid) v = ld_nc_v4(x + m * ld_x + g * 128 + hl * 8);
+    float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                  bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float s = __fdiv_rn(amax, 448.f);
+    if (valid) {
+      uint2 out;
+      out.x = cvt4_e4m3(quant_div(f[0], s), quant_div(f[1], s), quant_div(f[2], s), quant_div(f[3], s));
+      out.y = cvt4_e4m3(quant_div(f[4], s), quant_div(f[5], s), quant_div(f[6], s), quant_div(f[7], s));
+      *reinterpret_cast<uint2*>(q + m * K + g * 128 + hl * 8) = out;
+      if (hl == 0) scale[m * G + g] = s;
+    }
+  }
+}
+
+// One CTA (256 threads) per 128x128 block; thread t owns row t/2, 64 columns.
+__global__ void __launch_bounds__(256) quant_weight_kernel(const float* __restrict__ w, int64_t N, int64_t K,
+                                                           uint8_t* __restrict__ q, float* __restrict__ scale) {
+  const int64_t G = K / 128;
+  const int64_t nb = blockIdx.y;
+  const int64_t g = blockIdx.x;
+  const int t = threadIdx.x;
+  const int64_t row = nb * 128 + (t >> 1);
+  const int64_t col = g * 128 + (t & 1) * 64;
+  const bool valid = row < N;
+  float4 v[16];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    v[i] = valid ? __ldg(reinterpret_cast<const float4*>(w + row * K + col) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  __shared__ float red[8];
+  if ((t & 31) == 0) red[t >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  const float s = __fdiv_rn(amax, 448.f);
+  if (t == 0) scale[nb * G + g] = s;
+  if (!valid) return;
+  uint32_t packed[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    packed[i] = cvt4_e4m3(quant_div(v[i].x, s), quant_div(v[i].y, s), quant_div(v[i].z, s), quant_div(v[i].w, s));
+  uint4* dst = reinterpret_cast<uint4*>(q + row * K + col);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+}
+
+int launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q, float* scale, void* stream) {
+  const int64_t groups = M * (K / 128);
+  const int64_t need = (groups + 15) / 16;  // 16 groups per 256-thread block per pass
+  const int64_t cap = int64_t(device_sm_count()) * 8;
+  const int blocks = int(need < cap ? need : cap);
+  quant_act_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x), M, K, ld_x, static_cast<uint8_t*>(q), scale);
+  return int(cudaGetLastError());
+}
+
+int launch_quant_weight(const float* w, int64_t N, int64_t K, void* q, float* scale, void* stream) {
+  dim3 grid(unsigned(K / 128), unsigned((N + 127) / 128));
+  quant_weight_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(w, N, K, static_cast<uint8_t*>(q), scale);
+  return int(cudaGetLastError());
+}
+
+}  // namespace fp8bs

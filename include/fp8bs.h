@@ -1,0 +1,173 @@
+/*
+ * fp8bs -- a8w8 block-scaled FP8 GEMM for NVIDIA B200 (sm_100a): C ABI.
+ *
+ * Operation (the GEMM behind gemm_a8w8_blockscale in the pages
+ * [cookbook#8] "Why aiter#5069's measured -25% kernel win moved serving
+ * throughput by 0.0%" -- GLM-5.2-FP8 is block quantised with
+ * weight_block_size [128,128] and so takes gemm_a8w8_blockscale -- and
+ * [aiter#7752] "[Perf] Retune gfx942 Qwen3.8-27B a8w8 blockscale decode rows
+ * for cold weights", section "Kernel"):
+ *
+ *   out[m,n] = sum_g a_scale[m,g] * w_scale[n/128,g]
+ *                    * sum_{k = 128g .. 128g+127} A[m,k] * W[n,k]
+ *
+ * A and W hold OCP e4m3 ("e4m3fn") codes, one byte per element; A is
+ * quantised per token per 1x128 group of K, W per 128x128 block; scales are
+ * float32 (scale = amax / 448); accumulation is float32; out is bfloat16,
+ * rounded once (round to nearest even).
+ *
+ * Conventions shared by every entry point:
+ *  - All matrices are row-major with the reduction dimension K contiguous
+ *    ("NT"): A [M,K], W [N,K], out [M,N], a_scale [M, K/128],
+ *    w_scale [ceil(N/128), K/128]. Leading dimensions equal the row length
+ *    unless an ld argument says otherwise.
+ *  - Every pointer to matrix data is a DEVICE pointer, owned by the caller;
+ *    the library never allocates, frees or retains device memory. Device
+ *    pointers must be 16-byte aligned (FP8BS_ERR_ALIGNMENT otherwise).
+ *  - Every compute call is asynchronous on the given CUDA stream (a
+ *    cudaStream_t; NULL is the legacy default stream), performs no host
+ *    synchronisation and no allocation, and may be captured in a CUDA graph.
+ *  - Arguments are validated before anything is launched: an invalid call
+ *    returns a status other than FP8BS_OK and launches nothing. A launch
+ *    failure reported by the CUDA runtime returns FP8BS_ERR_CUDA.
+ *  - There is no CPU fallback: without a usable sm_100 device the compute
+ *    calls return FP8BS_ERR_CUDA or FP8BS_ERR_UNSUPPORTED.
+ *  - No C++ exception crosses this interface. All functions are thread-safe;
+ *    the dispatch table's counters are process-global atomics.
+ */
+#ifndef FP8BS_H
+#define FP8BS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, without pulling in the CUDA headers. */
+typedef struct CUstream_st* fp8bs_stream_t;
+
+typedef enum {
+  FP8BS_OK = 0,
+  FP8BS_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, K % 128 != 0, N % 16 != 0, ... */
+  FP8BS_ERR_UNSUPPORTED = 2, /* shape or device the library has no kernel for */
+  FP8BS_ERR_ALIGNMENT = 3,   /* a device pointer or leading dimension is not 16-byte aligned */
+  FP8BS_ERR_WORKSPACE = 4,   /* workspace missing or smaller than fp8bs_workspace_bytes() */
+  FP8BS_ERR_CUDA = 5,        /* the CUDA runtime reported an error at launch */
+  FP8BS_ERR_TIMEOUT = 6      /* a kernel gave up a bounded device-side wait (see fp8bs_get_device_status) */
+} fp8bs_status;
+
+/* Operation ids for the dispatch table and workspace sizing. */
+enum { FP8BS_OP_A8W8_BLOCKSCALE = 0, FP8BS_OP_BF16 = 1, FP8BS_NUM_OPS = 2 };
+
+/*
+ * Activation quantisation, per token per 1x128 group.
+ * For every row m and group g (K/128 groups):
+ *   amax = max |x[m, 128g .. 128g+127]|,  a_scale[m,g] = amax / 448 (IEEE fp32 division),
+ *   q[m,k] = e4m3_rn_satfinite(x[m,k] / a_scale[m,g])  (IEEE fp32 division, one rounding);
+ * a group with amax == 0 gets a_scale 0 and codes +-0 (0x00 / 0x80, the sign of x).
+ * x_bf16 : device, bf16 [M, ld_x] (row stride ld_x elements, ld_x >= K, ld_x % 8 == 0)
+ * q_e4m3 : device, e4m3 codes [M, K] (row stride K), written
+ * a_scale: device, float32 [M, K/128] (row stride K/128), written
+ * group  : must be 128.
+ * Result bit-identical to the CPU oracle (codes and scales).
+ */
+fp8bs_status fp8bs_quant_act_per_token_group(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x,
+                                             void* q_e4m3, float* a_scale, int group,
+                                             fp8bs_stream_t stream);
+
+/*
+ * Weight quantisation, per 128x128 block ([cookbook#8]: weight_block_size [128,128]).
+ * For every block (nb, g): amax over rows 128nb .. min(N,128nb+128)-1 and columns
+ * 128g .. 128g+127; w_scale[nb,g] = amax / 448; codes as for activations.
+ * w_f32  : device, float32 [N, K]; q_e4m3: device, e4m3 [N, K]; w_scale: device, float32
+ * [ceil(N/128), K/128]. A set-up step (not on the per-call path).
+ */
+fp8bs_status fp8bs_quant_weight_block128(const float* w_f32, int64_t N, int64_t K, void* q_e4m3,
+                                         float* w_scale, fp8bs_stream_t stream);
+
+/*
+ * The a8w8 block-scaled GEMM (formula at the top of this file).
+ * A_e4m3 [M,K], a_scale [M,K/128], W_e4m3 [N,K], w_scale [ceil(N/128),K/128],
+ * out_bf16 [M,N]: device pointers. Requires M,N,K > 0, K % 128 == 0, N % 16 == 0.
+ * workspace: device scratch of at least fp8bs_workspace_bytes(FP8BS_OP_A8W8_BLOCKSCALE, M, N, K)
+ * bytes (may be NULL when that is 0). It must be zero-filled once before its first
+ * use; every call leaves it zero-filled again (it holds split-K partial sums and
+ * self-resetting arrival counters), so one workspace serves any number of calls on
+ * one stream. Calls that may run concurrently need separate workspaces.
+ * The kernel is picked by the dispatch table (fp8bs_dispatch_lookup): a
+ * weight-streaming split-K kernel for small M, a tcgen05/TMEM tensor-core kernel
+ * fed by TMA otherwise. Results are deterministic (split-K partial sums are
+ * reduced in a fixed order) and within the float32-accumulation bound of the
+ * float64 oracle rounded once to bf16.
+ */
+fp8bs_status fp8bs_gemm_a8w8_blockscale(const void* A_e4m3, const float* a_scale, const void* W_e4m3,
+                                        const float* w_scale, void* out_bf16, int64_t M, int64_t N,
+                                        int64_t K, void* workspace, size_t workspace_bytes,
+                                        fp8bs_stream_t stream);
+
+/*
+ * Companion bf16 GEMM for the small-N router / indexer projections ([cookbook#8]:
+ * the live BF16 lookups are the MoE router and the DSA indexer's weights_proj;
+ * [aiter#7247] "Technical Details": N = 32..1024, some with fp32 output).
+ * out[m,n] = sum_k A[m,k] * W[n,k], float32 accumulation, rounded once to bf16,
+ * or stored as float32 when out_is_fp32 != 0.
+ * A [M,K] bf16, W [N,K] bf16, out [M,N]: device. Requires K % 64 == 0, N % 16 == 0.
+ * workspace as for fp8bs_gemm_a8w8_blockscale (op FP8BS_OP_BF16).
+ */
+fp8bs_status fp8bs_gemm_bf16(const void* A_bf16, const void* W_bf16, void* out, int out_is_fp32,
+                             int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                             fp8bs_stream_t stream);
+
+/* Bytes of workspace a call of op with this shape needs (0 if none). Host only. */
+size_t fp8bs_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
+
+/*
+ * Dispatch table ([aiter#7752] "PR-specific question": the lookup probes exact M,
+ * then the next power of two below 16 or the next multiple of 16 up to 256, then
+ * the next power of two; [mi210 docs/43] section 6: a miss runs the per-shape
+ * default kernel). Rows are keyed (op, padded_M, N, K). Every lookup made by a GEMM
+ * call is counted; fp8bs_dispatch_lookup with record=0 only inspects.
+ * padded_M: the row's M on a hit, 0 on a miss. cfg: the kernel configuration name
+ * that runs (NUL-terminated, truncated to cfg_len).
+ */
+fp8bs_status fp8bs_dispatch_lookup(int op, int64_t M, int64_t N, int64_t K, int record,
+                                   int64_t* padded_M, int* hit, char* cfg, size_t cfg_len);
+
+/* Add or replace a table row: kernel configuration cfg (a name returned by
+ * fp8bs_dispatch_list_configs) for (op, M, N, K). */
+fp8bs_status fp8bs_dispatch_set_row(int op, int64_t M, int64_t N, int64_t K, const char* cfg);
+
+/* Remove all rows (keep_builtin = 0) or restore the built-in rows (keep_builtin = 1). */
+fp8bs_status fp8bs_dispatch_reset_table(int keep_builtin);
+
+/* Newline-separated list of the kernel configuration names a row may name for op. */
+fp8bs_status fp8bs_dispatch_list_configs(int op, char* buf, size_t len);
+
+/* Lookup counters for op since the last fp8bs_dispatch_reset_stats: all lookups
+ * (hits, misses) and distinct keys (M, N, K, padded_M, cfg) among them. */
+fp8bs_status fp8bs_dispatch_stats(int op, uint64_t* hits, uint64_t* misses, uint64_t* distinct_hits,
+                                  uint64_t* distinct_misses);
+fp8bs_status fp8bs_dispatch_reset_stats(void);
+
+/* Census: one JSON object per distinct lookup key with its count, as a JSON array. */
+fp8bs_status fp8bs_dispatch_dump_json(char* buf, size_t len);
+
+/* 64-bit FNV-1a hash of the current table rows (identifies the table that ran). */
+uint64_t fp8bs_dispatch_table_hash(void);
+
+/* Synchronises the stream, then reports and clears the device-side status word:
+ * FP8BS_ERR_TIMEOUT if any kernel abandoned a bounded wait since the last call. */
+fp8bs_status fp8bs_get_device_status(fp8bs_stream_t stream);
+
+const char* fp8bs_status_string(fp8bs_status status);
+
+/* Library version string. */
+const char* fp8bs_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BS_H */

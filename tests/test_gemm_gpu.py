@@ -1,0 +1,165 @@
+"""a8w8 block-scale GEMM kernels vs the oracle (both kernel paths, tails, exact cases,
+determinism, graph replay, full-size configurations on sampled rows)."""
+
+import numpy as np
+import pytest
+import torch
+
+import fp8_block_scaled_a8w8_b200 as fb
+from fp8_block_scaled_a8w8_b200 import inputs
+from oracle import gemm as ogemm
+from oracle import quant as oquant
+from tests.helpers import bf16_bits, check_a8w8, codes_from_device, codes_to_device
+
+pytestmark = pytest.mark.gpu
+OP = fb.OP_A8W8_BLOCKSCALE
+
+
+def _raw_case(M, N, K, seed):
+    A_q = inputs.random_e4m3_codes((M, K), seed)
+    W_q = inputs.random_e4m3_codes((N, K), seed + 1)
+    a_s = inputs.random_scales((M, K // 128), seed + 2)
+    w_s = inputs.random_scales(((N + 127) // 128, K // 128), seed + 3)
+    return A_q, a_s, W_q, w_s
+
+
+def _run(A_q, a_s, W_q, w_s, cfg=None):
+    M, K = A_q.shape
+    N = W_q.shape[0]
+    if cfg is not None:
+        fb.dispatch_set_row(OP, M, N, K, cfg)
+    try:
+        y = fb.gemm_a8w8_blockscale(codes_to_device(A_q), torch.from_numpy(a_s).cuda(), codes_to_device(W_q),
+                                    torch.from_numpy(w_s).cuda())
+        torch.cuda.synchronize()
+        assert fb.get_device_status() == 0
+    finally:
+        if cfg is not None:
+            fb.dispatch_reset_table(True)
+    return y
+
+
+GEMV_SHAPES = [(16, 128), (128, 256), (272, 640), (1040, 1152)]
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 9, 13, 16, 17, 24, 31, 32])
+@pytest.mark.parametrize("N,K", GEMV_SHAPES)
+def test_gemv_path_parity(M, N, K):
+    case = _raw_case(M, N, K, seed=M * 1000 + N + K)
+    _, cfg = fb.dispatch_lookup(OP, M, N, K)
+    assert cfg.startswith("a8w8_gemv")
+    check_a8w8(_run(*case), *case)
+
+
+@pytest.mark.parametrize("cfg", ["a8w8_gemv_d2", "a8w8_gemv_d3", "a8w8_gemv_d4"])
+@pytest.mark.parametrize("M", [1, 7, 16, 25])
+def test_gemv_depths(cfg, M):
+    case = _raw_case(M, 400, 1408, seed=M + 77)
+    check_a8w8(_run(*case, cfg=cfg), *case)
+
+
+TC_SHAPES = [(256, 512), (384, 1024), (1280, 768)]
+
+
+@pytest.mark.parametrize("M", [33, 100, 128, 129, 255, 300])
+@pytest.mark.parametrize("N,K", TC_SHAPES)
+def test_tc_path_parity(M, N, K):
+    case = _raw_case(M, N, K, seed=M * 31 + N + K)
+    _, cfg = fb.dispatch_lookup(OP, M, N, K)
+    assert cfg.startswith("a8w8_tc")
+    check_a8w8(_run(*case), *case)
+
+
+@pytest.mark.parametrize("cfg", ["a8w8_tc_bn128", "a8w8_tc_bn256"])
+@pytest.mark.parametrize("M,N,K", [(1, 256, 128), (40, 512, 2048), (300, 1536, 640), (2, 272, 256)])
+def test_tc_configs_any_m(cfg, M, N, K):
+    """The tensor-core kernel on any M, including tiny M and N tails (a row can name it)."""
+    case = _raw_case(M, N, K, seed=M + N + K)
+    check_a8w8(_run(*case, cfg=cfg), *case)
+
+
+@pytest.mark.parametrize("M,N,K,cfg", [(3, 272, 512, None), (16, 1024, 1024, None), (200, 512, 1024, None),
+                                       (130, 384, 512, "a8w8_tc_bn128"), (64, 512, 384, "a8w8_tc_bn256")])
+def test_integer_valued_bit_exact(M, N, K, cfg):
+    """Integer e4m3 values |v| <= 4 and power-of-two scales: every partial sum is exact,
+    so the bf16 output must equal bf16(exact) bit for bit."""
+    rng = np.random.default_rng(M + N)
+    codes = np.array([0x00, 0x38, 0x40, 0x44, 0x48], dtype=np.uint8)  # 0, 1, 2, 3, 4
+    A_q = codes[rng.integers(0, 5, (M, K))] | (rng.integers(0, 2, (M, K)) << 7).astype(np.uint8)
+    W_q = codes[rng.integers(0, 5, (N, K))] | (rng.integers(0, 2, (N, K)) << 7).astype(np.uint8)
+    a_s = np.ldexp(1.0, rng.integers(-6, 3, (M, K // 128))).astype(np.float32)
+    w_s = np.ldexp(1.0, rng.integers(-6, 3, ((N + 127) // 128, K // 128))).astype(np.float32)
+    y = _run(A_q, a_s, W_q, w_s, cfg)
+    _, ref_bf16 = ogemm.gemm_a8w8_blockscale(A_q, a_s, W_q, w_s)
+    assert np.array_equal(y.float().cpu().numpy().astype(np.float64), ref_bf16)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 5120, 6144), (9, 2048, 1024), (700, 1024, 1024)])
+def test_deterministic_and_graph_replay(M, N, K):
+    case = _raw_case(M, N, K, seed=3)
+    A, a_s, W, w_s = (codes_to_device(case[0]), torch.from_numpy(case[1]).cuda(), codes_to_device(case[2]),
+                      torch.from_numpy(case[3]).cuda())
+    y1 = fb.gemm_a8w8_blockscale(A, a_s, W, w_s)
+    y2 = fb.gemm_a8w8_blockscale(A, a_s, W, w_s)
+    out = torch.empty_like(y1)
+    ws = torch.zeros(max(fb.workspace_bytes(OP, M, N, K), 256), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        fb.gemm_a8w8_blockscale(A, a_s, W, w_s, out=out, workspace=ws)
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(bf16_bits(out), bf16_bits(y1))
+    assert np.array_equal(bf16_bits(y1), bf16_bits(y2))
+    check_a8w8(y1, *case)
+
+
+def test_config0_end_to_end():
+    """M=1, N=5120, K=6144, seed 0: bf16 activations and float32 weights quantised on the
+    GPU, then the GEMM; the oracle quantises and multiplies on its own."""
+    x, w = inputs.config0(0)
+    q, s = fb.quant_act_per_token_group(x.cuda())
+    wq, ws = fb.quant_weight_block128(w.cuda())
+    y = fb.gemm_a8w8_blockscale(q, s, wq, ws)
+    torch.cuda.synchronize()
+    A_q, a_s = oquant.quant_act_per_token_group(x.float().numpy())
+    W_q, w_s = oquant.quant_weight_block128(w.numpy())
+    rl, rl_bf16 = check_a8w8(y, A_q, a_s, W_q, w_s)
+    assert rl < 2.2e-3  # the bf16 output-rounding floor the pages report is 1.7e-3
+
+
+@pytest.mark.parametrize("nk_index", [0, 1, 2, 3])
+def test_decode_sweep_full_size(nk_index):
+    N, K = inputs.DECODE_NK[nk_index]
+    w = inputs.weight_f32(N, K, inputs.decode_seed_w(nk_index))
+    wq, ws = fb.quant_weight_block128(w.cuda())
+    W_q, w_s = oquant.quant_weight_block128(w.numpy())
+    assert np.array_equal(codes_from_device(wq), W_q)
+    for mi, M in enumerate(inputs.DECODE_MS):
+        x = inputs.activation_bf16(M, K, inputs.decode_seed_a(nk_index, mi))
+        q, s = fb.quant_act_per_token_group(x.cuda())
+        y = fb.gemm_a8w8_blockscale(q, s, wq, ws)
+        torch.cuda.synchronize()
+        A_q, a_s = oquant.quant_act_per_token_group(x.float().numpy())
+        check_a8w8(y, A_q, a_s, W_q, w_s)
+
+
+@pytest.mark.parametrize("M", [2048, 6016, 8192])
+def test_prefill_full_size_sampled_rows(M):
+    N, K = inputs.PREFILL_NK[1]  # (34816, 5120)
+    w = inputs.weight_f32(N, K, 11)
+    x = inputs.activation_bf16(M, K, 12 + M, outliers=True)
+    wq, ws = fb.quant_weight_block128(w.cuda())
+    q, s = fb.quant_act_per_token_group(x.cuda())
+    y = fb.gemm_a8w8_blockscale(q, s, wq, ws)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(M)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1, M - 2, (M // 128) * 128 - 1],
+                                     rng.choice(M, 9, replace=False)]))
+    rows = rows[rows < M]
+    W_q, w_s = oquant.quant_weight_block128(w.numpy())
+    A_q, a_s = oquant.quant_act_per_token_group(x.float().numpy()[rows])
+    check_a8w8(y.cpu()[torch.from_numpy(rows)], A_q, a_s, W_q, w_s)
