@@ -1,0 +1,467 @@
+"""Benchmark: a8w8 block-scale GEMM, us/call, TFLOPS and HBM GB/s on cold weights vs roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Default workload (N=1): the decode sweep -- M in {1,2,3,4,8,9,16} on the four
+Qwen3.8-27B projections (N,K) = (5120,6144), (14336,5120), (16384,5120),
+(34816,5120) of [aiter#7752] "Kernel". One step is one pass of the hot path over
+the sweep: for each of the 28 (M,N,K) calls, per-token 1x128 activation
+quantisation, dispatch, and the block-scaled GEMM. Weights are quantised once
+(set-up) and rotated over >= 512 MiB of distinct device copies per shape, so every
+call reads cold weights from HBM ([vllm#1065]: a 48 MiB rotation was 19%
+optimistic, 512 MiB within 1.1% of in-model timing). The working set of every
+step is far above the 126 MB L2, which replaces an L2 flush between steps.
+
+Each step is captured once in a CUDA graph (one graph per rotation phase) and
+replayed; CUDA events recorded inside the graphs time every GEMM launch. The
+timed region is bracketed by a barrier and a device synchronise on both sides and
+the step time is the max over ranks. N>1 runs N independent replicas (the path
+has no exchange step).
+
+--impl reference times the CPU oracle (the only other arm this build has) on a
+bounded sample of the same workload, on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from fp8_block_scaled_a8w8_b200 import inputs  # noqa: E402
+
+METRIC = "a8w8 blockscale GEMM µs/call, TFLOPS & HBM GB/s (cold weights) vs roofline"
+ROTATE_BYTES = int(os.environ.get("FP8BS_ROTATE_MIB", "512")) * (1 << 20)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def a8w8_bytes(M, N, K):
+    """Algorithmic bytes of one call: A + a_scale + W + w_scale + out."""
+    G = K // 128
+    return M * K + 4 * M * G + N * K + 4 * ((N + 127) // 128) * G + 2 * M * N
+
+
+def bf16_bytes(M, N, K, out_fp32):
+    return 2 * M * K + 2 * N * K + (4 if out_fp32 else 2) * M * N
+
+
+def workload_calls(name):
+    """List of (M, N, K, nk_index, m_index, outliers) for the workload."""
+    if name == "decode_sweep":
+        return [(M, N, K, i, j, False) for i, (N, K) in enumerate(inputs.DECODE_NK) for j, M in enumerate(inputs.DECODE_MS)]
+    if name == "decode_m1_n5120_k6144":
+        return [(1, 5120, 6144, 0, 0, False)]
+    if name == "prefill":
+        return [(M, N, K, i, j, True) for i, (N, K) in enumerate(inputs.PREFILL_NK) for j, M in enumerate(inputs.PREFILL_MS)]
+    if name == "ladder":
+        N, K = inputs.LADDER_NK
+        return [(M, N, K, 0, j, False) for j, M in enumerate(inputs.ladder_ms())]
+    raise SystemExit(f"unknown workload {name}")
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(parts)
+            except ValueError:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        load = sorted(sm)[len(sm) // 2:] if sm else []  # upper half: samples under load
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(load)) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import fp8_block_scaled_a8w8_b200 as fb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    fb.lib()
+    pk = peaks()
+
+    calls = workload_calls(args.workload)
+    uses = {}
+    for (M, N, K, i, j, o) in calls:
+        uses[(N, K)] = uses.get((N, K), 0) + 1
+
+    # ---- set-up (untimed): weights quantised on the GPU, rotated copies, activations
+    wcopies = {}
+    for (N, K), u in uses.items():
+        nk_index = [nk for (_, n, k, nk, _, _) in calls if (n, k) == (N, K)][0]
+        w = inputs.weight_f32(N, K, inputs.decode_seed_w(nk_index)).to(dev)
+        wq, ws = fb.quant_weight_block128(w)
+        del w
+        per = N * K + ws.numel() * 4
+        n = max(1, math.ceil(ROTATE_BYTES / per))
+        n = u * math.ceil(n / u)  # a multiple of the uses per step: every step has the same period
+        copies = [(wq, ws)] + [(wq.clone(), ws.clone()) for _ in range(n - 1)]
+        wcopies[(N, K)] = copies
+    torch.cuda.synchronize()
+
+    # activations: one seeded base per shape (rows = largest M of that shape), calls take row
+    # slices; quantised activations and outputs likewise share one buffer per shape (calls run
+    # in stream order)
+    maxm = {}
+    for (M, N, K, i, j, o) in calls:
+        maxm[(N, K)] = max(maxm.get((N, K), 0), M)
+    bx, bq, bs, bo = {}, {}, {}, {}
+    for (N, K), mm in maxm.items():
+        i, o = [(ci, co) for (_, n, k, ci, _, co) in calls if (n, k) == (N, K)][0]
+        bx[(N, K)] = inputs.activation_bf16(mm, K, inputs.decode_seed_a(i, 0), outliers=o).to(dev)
+        bq[(N, K)] = torch.empty((mm, K), dtype=torch.float8_e4m3fn, device=dev)
+        bs[(N, K)] = torch.empty((mm, K // 128), dtype=torch.float32, device=dev)
+        bo[(N, K)] = torch.empty((mm, N), dtype=torch.bfloat16, device=dev)
+    xs = [bx[(N, K)][:M] for (M, N, K, *_r) in calls]
+    qs = [bq[(N, K)][:M] for (M, N, K, *_r) in calls]
+    ss = [bs[(N, K)][:M] for (M, N, K, *_r) in calls]
+    outs = [bo[(N, K)][:M] for (M, N, K, *_r) in calls]
+    ws_bytes = max(fb.workspace_bytes(fb.OP_A8W8_BLOCKSCALE, M, N, K) for (M, N, K, *_r) in calls)
+    workspace = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    cfgs = [fb.dispatch_lookup(fb.OP_A8W8_BLOCKSCALE, M, N, K)[1] for (M, N, K, *_r) in calls]
+
+    # rotation phase: step s, call c uses copy (s * uses + rank_of_c_within_shape) % n_copies
+    period = 1
+    for (N, K), u in uses.items():
+        n = len(wcopies[(N, K)])
+        period = period * (n // u) // math.gcd(period, n // u)
+
+    stream = torch.cuda.Stream(device=dev)
+    n_calls = len(calls)
+
+    def step_launches(s, ev=None):
+        ctr = {}
+        for c, (M, N, K, *_r) in enumerate(calls):
+            k = ctr.get((N, K), 0)
+            ctr[(N, K)] = k + 1
+            cp = wcopies[(N, K)]
+            wq, wsc = cp[(s * uses[(N, K)] + k) % len(cp)]
+            fb.quant_act_per_token_group(xs[c], q=qs[c], scale=ss[c], stream=stream)
+            if ev is not None:
+                ev[c][0].record(stream)
+            fb.gemm_a8w8_blockscale(qs[c], ss[c], wq, wsc, out=outs[c], workspace=workspace, stream=stream)
+            if ev is not None:
+                ev[c][1].record(stream)
+
+    # events inside the graphs: one pair per GEMM launch per phase
+    events = [[[torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True)]
+               for _ in range(n_calls)] for _ in range(period)]
+    graphs = []
+    fb.dispatch_reset_stats()
+    with torch.cuda.stream(stream):
+        for ph in range(period):  # eager warm-up of each phase (also loads modules)
+            step_launches(ph)
+        stream.synchronize()
+        for ph in range(period):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step_launches(ph, events[ph])
+            graphs.append(g)
+    torch.cuda.synchronize()
+    census = fb.dispatch_stats(fb.OP_A8W8_BLOCKSCALE)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for s in range(args.warmup):
+        graphs[s % period].replay()
+    barrier()
+
+    clocks = ClockSampler(dev.index)
+    if rank == 0:
+        clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    gemm_ms = np.zeros(n_calls)
+    barrier()
+    t_start.record(stream)
+    for s in range(args.steps):
+        with torch.cuda.stream(stream):
+            graphs[(args.warmup + s) % period].replay()
+        # per-launch GEMM durations: read back lazily after the region (events of the last
+        # replay of each phase hold their last timestamps)
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop() if rank == 0 else None
+    step_ms = t_start.elapsed_time(t_end) / args.steps
+
+    # per-launch GEMM times of the last replay of every phase
+    per_phase = []
+    last = {}
+    for s in range(args.steps):
+        last[(args.warmup + s) % period] = True
+    for ph in last:
+        per_phase.append([events[ph][c][0].elapsed_time(events[ph][c][1]) for c in range(n_calls)])
+    gemm_ms = np.mean(np.array(per_phase), axis=0)
+
+    t = torch.tensor([step_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms = float(t.item())
+
+    # ---- end to end through the public API: pinned host inputs in, results out, per step
+    e2e = None
+    e2e_steps = args.e2e_steps if n_calls <= 64 and max(maxm.values()) <= 64 else min(args.e2e_steps, 3)
+    if e2e_steps > 0:
+        hx = [x.cpu().pin_memory() for x in xs]
+        hy = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        dxb = {k: torch.empty_like(v) for k, v in bx.items()}
+        dx = [dxb[(N, K)][:M] for (M, N, K, *_r) in calls]
+        h2d = sum(x.numel() * x.element_size() for x in xs)
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+
+        def e2e_step(s):
+            with torch.cuda.stream(stream):
+                ctr = {}
+                for c, (M, N, K, *_r) in enumerate(calls):
+                    dx[c].copy_(hx[c], non_blocking=True)
+                    k = ctr.get((N, K), 0)
+                    ctr[(N, K)] = k + 1
+                    cp = wcopies[(N, K)]
+                    wq, wsc = cp[(s * uses[(N, K)] + k) % len(cp)]
+                    q, sc = fb.quant_act_per_token_group(dx[c], q=qs[c], scale=ss[c], stream=stream)
+                    fb.gemm_a8w8_blockscale(q, sc, wq, wsc, out=outs[c], workspace=workspace, stream=stream)
+                    hy[c].copy_(outs[c], non_blocking=True)
+        for s in range(3):
+            e2e_step(s)
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(e2e_steps):
+            e2e_step(s)
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1) / e2e_steps
+        te = torch.tensor([e2e_ms], device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item())
+        e2e = {"value": round(e2e_ms * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "api": "fp8_block_scaled_a8w8_b200.quant_act_per_token_group + gemm_a8w8_blockscale (eager)"}
+
+    if rank == 0:
+        detail = []
+        tot_bytes = 0.0
+        tot_ms = 0.0
+        for c, (M, N, K, *_r) in enumerate(calls):
+            by = a8w8_bytes(M, N, K)
+            fl = 2.0 * M * N * K
+            us = gemm_ms[c] * 1000.0
+            roof_us = max(by / (pk["hbm_gbs"] * 1e3), fl / (2 * pk["bf16_tflops"] * 1e6))
+            detail.append({"M": M, "N": N, "K": K, "cfg": cfgs[c], "us": round(us, 3),
+                           "GBps": round(by / us / 1e3, 1), "TFLOPS": round(fl / us / 1e6, 2),
+                           "roofline_frac": round(roof_us / us, 3)})
+            tot_bytes += by
+            tot_ms += gemm_ms[c]
+        tot_flops = sum(2.0 * M * N * K for (M, N, K, *_r) in calls)
+        fp8_peak = 2.0 * pk["bf16_tflops_sustained"]  # fp8 dense = 2x bf16 (nominal 4.5 / 2.25 PFLOP/s)
+        hbm_bound = tot_bytes / (pk["hbm_gbs"] * 1e9) >= tot_flops / (fp8_peak * 1e12)
+        if hbm_bound:
+            achieved = tot_bytes / (tot_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(achieved / pk["hbm_gbs"], 4),
+                    "peak_source": f"{pk['source']} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"}
+        else:
+            achieved = tot_flops / (tot_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(achieved / fp8_peak, 4),
+                    "peak_source": f"2 x {pk['source']} sustained bf16 cuBLAS (fp8/bf16 nominal ratio 2)"}
+        roof["traffic"] = None
+        roof["kernel"] = "gemm_a8w8_blockscale: " + ", ".join(sorted(set(cfgs)))
+        roof["algorithmic_bytes_per_step"] = int(tot_bytes)
+        roof["gemm_us_per_step"] = round(tot_ms * 1000.0, 2)
+        cpu = cpu_baseline(args.workload) if (args.cpu_baseline and world == 1) else None
+        line = {
+            "metric": METRIC, "value": round(step_ms * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 -> bf16",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no dataset)",
+            "config": {"workload": args.workload, "description": inputs.WORKLOADS[args.workload], "calls_per_step": n_calls,
+                       "weight_rotation_mib": ROTATE_BYTES >> 20,
+                       "l2": "working set per step >> 126 MB L2 (rotated weights); no flush needed",
+                       "parallelism": f"replicas x{world}", "timing": "CUDA graphs replayed, CUDA events, max over ranks"},
+            "roofline": roof,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * n_calls * args.steps,
+            "clocks": clk, "dispatch": {**census, "table_hash": fb.dispatch_table_hash()},
+            "detail": detail,
+        }
+        print(json.dumps(line), flush=True)
+    for g in graphs:
+        del g
+    graphs.clear()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def _oracle_call(M, N, K, i, j, o, wcache):
+    from oracle import gemm as ogemm, quant as oquant
+    key = (N, K)
+    if key not in wcache:
+        w = inputs.weight_f32(N, K, inputs.decode_seed_w(i)).numpy()
+        wcache[key] = oquant.quant_weight_block128(w)  # set-up, untimed
+    x = inputs.activation_bf16(M, K, inputs.decode_seed_a(i, j), outliers=o).float().numpy()
+    W_q, w_s = wcache[key]
+    t0 = time.perf_counter()
+    A_q, a_s = oquant.quant_act_per_token_group(x)
+    ogemm.gemm_a8w8_blockscale(A_q, a_s, W_q, w_s)
+    return time.perf_counter() - t0
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(workload, budget_s=20.0):
+    """The oracle as it stands, timed on the host on a bounded sample of the workload."""
+    calls = workload_calls(workload)
+    rng = np.random.default_rng(0)
+    order = list(rng.permutation(len(calls)))
+    wcache = {}
+    spent, n, done = 0.0, 0, []
+    for c in order:
+        M, N, K, i, j, o = calls[c]
+        if workload in ("prefill", "ladder") and M > 64:
+            M = 64  # rows of a large-M call: the oracle is row-separable; time per row is scaled below
+        dt = _oracle_call(M, N, K, i, j, o, wcache)
+        scale = calls[c][0] / M
+        spent += dt
+        done.append(dt * scale)
+        n += 1
+        if spent > budget_s:
+            break
+    us = float(np.mean(done)) * 1e6
+    return {"value": round(us, 1), "unit": "µs/call", "cores": _threads(), "kind": "oracle",
+            "sample": f"{n} of {len(calls)} calls of the {workload} workload (random order), quant + GEMM in float64"
+                      f"{'; large-M calls timed on 64 rows and scaled by M/64' if workload in ('prefill', 'ladder') else ''}"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and rank != 0:
+        return
+    calls = workload_calls(args.workload)
+    wcache = {}
+    for s in range(args.warmup):
+        M, N, K, i, j, o = calls[s % len(calls)]
+        _oracle_call(min(M, 64), N, K, i, j, o, wcache)
+    times = []
+    for s in range(args.steps):
+        M, N, K, i, j, o = calls[(args.warmup + s) % len(calls)]
+        m = min(M, 64)
+        times.append(_oracle_call(m, N, K, i, j, o, wcache) * M / m)
+    us = float(np.mean(times)) * 1e6
+    cores = _threads()
+    line = {"impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "µs/call", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1000.0, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "description": inputs.WORKLOADS[args.workload]},
+            "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": cores, "kind": "oracle",
+                             "sample": f"one call per step, cycling through the {args.workload} calls"},
+            "e2e": {"value": round(us, 1), "unit": "µs/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode_sweep", choices=list(inputs.WORKLOADS))
+    ap.add_argument("--impl", default="fp8bs", choices=["fp8bs", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -11,7 +11,8 @@
 // A warp that covers a whole 16-row tile writes its output directly; a tile shared by
 // several warps is finished by the last one to arrive (an atomic counter per tile), which
 // sums the others' float32 partials in warp order -- a fixed order, so results are
-// bit-reproducible -- writes the output and resets the counter to zero for the next call.
+// bit-reproducible -- writes the output, and zeroes the partials it read and the tile's
+// counter, so the whole workspace is zero-filled again when the kernel ends.
 //
 // Math: swap-AB mma.sync.m16n8k32 (e4m3 -> f32): 16 W rows are the MMA's M, up to 8
 // tokens its N. Inside one MMA the 32 k positions may be matched between A and B in any
@@ -47,11 +48,6 @@ struct GemvArgs {
   float* part;             // [2 * n_active_warps][NB * 4 * 32]
   unsigned* counter;       // [N / 16]
   int out_fp32;
-};
-
-template <bool kFp8>
-struct Unit {
-  uint4 wa[2], wb[2];  // W rows gid / gid+8, chunks c = 0, 1
 };
 
 __device__ __forceinline__ int64_t warp_of_unit(int64_t u, int64_t U, int64_t W) { return ((u + 1) * W - 1) / U; }
@@ -214,11 +210,14 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs p) {
               for (int64_t ww = wf; ww <= wl; ++ww) {
                 const int ft = int((U * ww / Wn) / G);
                 const int sl = 2 * int(ww) + (t == ft ? 0 : 1);
-                const float* src = p.part + int64_t(sl) * (NB * 4 * 32);
+                float* src = p.part + int64_t(sl) * (NB * 4 * 32);
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-                  for (int i = 0; i < 4; ++i) sum[nb][i] += __ldcg(src + (nb * 4 + i) * 32 + lane);
+                  for (int i = 0; i < 4; ++i) {
+                    sum[nb][i] += __ldcg(src + (nb * 4 + i) * 32 + lane);
+                    __stcg(src + (nb * 4 + i) * 32 + lane, 0.f);  // leave the workspace zero-filled
+                  }
               }
               store_out<kFp8, NB>(p, t, lane, sum);
               if (lane == 0) p.counter[t] = 0u;

@@ -163,3 +163,18 @@ def test_prefill_full_size_sampled_rows(M):
     W_q, w_s = oquant.quant_weight_block128(w.numpy())
     A_q, a_s = oquant.quant_act_per_token_group(x.float().numpy()[rows])
     check_a8w8(y.cpu()[torch.from_numpy(rows)], A_q, a_s, W_q, w_s)
+
+
+def test_workspace_left_zero_and_shared_across_shapes():
+    """Every call leaves its workspace zero-filled, so calls of different shapes can share
+    one workspace in stream order."""
+    shapes = [(1, 5120, 6144), (16, 34816, 5120), (9, 2048, 1024), (3, 14336, 5120), (1, 5120, 6144)]
+    need = max(fb.workspace_bytes(OP, *s) for s in shapes)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for i, (M, N, K) in enumerate(shapes):
+        case = _raw_case(M, N, K, seed=100 + i)
+        y = fb.gemm_a8w8_blockscale(codes_to_device(case[0]), torch.from_numpy(case[1]).cuda(),
+                                    codes_to_device(case[2]), torch.from_numpy(case[3]).cuda(), workspace=ws)
+        torch.cuda.synchronize()
+        assert int(ws.count_nonzero()) == 0
+        check_a8w8(y, *case)

@@ -28,7 +28,7 @@ def test_act_quant_edge_groups():
     x = torch.zeros((5, K), dtype=torch.float32)
     x[1, :128] = -0.0                                     # all -0 group
     x[2, 5] = 3.0                                         # single nonzero
-    x[3, :] = torch.linspace(-3e38, 3e38, K)              # huge values
+    x[3, :] = torch.linspace(-3e38, 3e38, K, dtype=torch.float64).float()  # huge finite values
     x[4, 128:256] = 2.0 ** -133                           # bf16 subnormals
     x[4, 300] = -(2.0 ** -130)
     x[0, 640:768] = torch.tensor([2.0 ** (i % 20 - 10) * (-1) ** i for i in range(128)])
