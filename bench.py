@@ -62,8 +62,11 @@ def bf16_bytes(M, N, K, out_fp32):
     return 2 * M * K + 2 * N * K + (4 if out_fp32 else 2) * M * N
 
 
-def workload_calls(name):
+def workload_calls(name, shape=None):
     """List of (M, N, K, nk_index, m_index, outliers) for the workload."""
+    if shape:
+        M, N, K = (int(v) for v in shape.split(","))
+        return [(M, N, K, 0, 0, False)]
     if name == "decode_sweep":
         return [(M, N, K, i, j, False) for i, (N, K) in enumerate(inputs.DECODE_NK) for j, M in enumerate(inputs.DECODE_MS)]
     if name == "decode_m1_n5120_k6144":
@@ -153,7 +156,7 @@ def run_gpu(args):
     fb.lib()
     pk = peaks()
 
-    calls = workload_calls(args.workload)
+    calls = workload_calls(args.workload, args.shape)
     uses = {}
     for (M, N, K, i, j, o) in calls:
         uses[(N, K)] = uses.get((N, K), 0) + 1
@@ -203,22 +206,26 @@ def run_gpu(args):
     n_calls = len(calls)
 
     def step_launches(s, ev=None):
+        """One step: the 28 activation quantisations, then the 28 GEMMs back to back (the
+        calls are independent, so the GEMMs run consecutively and programmatic dependent
+        launch overlaps each one's tail with the next one's weight stream)."""
+        for c in range(n_calls):
+            fb.quant_act_per_token_group(xs[c], q=qs[c], scale=ss[c], stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
         ctr = {}
         for c, (M, N, K, *_r) in enumerate(calls):
             k = ctr.get((N, K), 0)
             ctr[(N, K)] = k + 1
             cp = wcopies[(N, K)]
             wq, wsc = cp[(s * uses[(N, K)] + k) % len(cp)]
-            fb.quant_act_per_token_group(xs[c], q=qs[c], scale=ss[c], stream=stream)
-            if ev is not None:
-                ev[c][0].record(stream)
-            fb.gemm_a8w8_blockscale(qs[c], ss[c], wq, wsc, out=outs[c], workspace=workspace, stream=stream)
-            if ev is not None:
-                ev[c][1].record(stream)
+            fb.gemm_a8w8_blockscale(qs[c], ss[c], wq, wsc, out=outs[c], workspace=workspace, stream=stream,
+                                    static_weights=True)
+        if ev is not None:
+            ev[1].record(stream)
 
-    # events inside the graphs: one pair per GEMM launch per phase
-    events = [[[torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True)]
-               for _ in range(n_calls)] for _ in range(period)]
+    # events inside the graphs: around the block of GEMM launches of each phase
+    events = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(period)]
     graphs = []
     fb.dispatch_reset_stats()
     with torch.cuda.stream(stream):
@@ -238,8 +245,9 @@ def run_gpu(args):
             dist.barrier()
         torch.cuda.synchronize()
 
-    for s in range(args.warmup):
-        graphs[s % period].replay()
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            graphs[s % period].replay()
     barrier()
 
     clocks = ClockSampler(dev.index)
@@ -247,27 +255,20 @@ def run_gpu(args):
         clocks.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    gemm_ms = np.zeros(n_calls)
     barrier()
     t_start.record(stream)
     for s in range(args.steps):
         with torch.cuda.stream(stream):
             graphs[(args.warmup + s) % period].replay()
-        # per-launch GEMM durations: read back lazily after the region (events of the last
-        # replay of each phase hold their last timestamps)
     t_end.record(stream)
     barrier()
     clk = clocks.stop() if rank == 0 else None
     step_ms = t_start.elapsed_time(t_end) / args.steps
 
-    # per-launch GEMM times of the last replay of every phase
-    per_phase = []
-    last = {}
-    for s in range(args.steps):
-        last[(args.warmup + s) % period] = True
-    for ph in last:
-        per_phase.append([events[ph][c][0].elapsed_time(events[ph][c][1]) for c in range(n_calls)])
-    gemm_ms = np.mean(np.array(per_phase), axis=0)
+    # average GEMM launch duration: the GEMM block of the last replay of every phase
+    gemm_block_ms = [events[ph][0].elapsed_time(events[ph][1]) for ph in sorted(
+        {(args.warmup + s) % period for s in range(args.steps)})]
+    gemm_ms_per_call = float(np.mean(gemm_block_ms)) / n_calls
 
     t = torch.tensor([step_ms], device=dev)
     if world > 1:
@@ -295,7 +296,8 @@ def run_gpu(args):
                     cp = wcopies[(N, K)]
                     wq, wsc = cp[(s * uses[(N, K)] + k) % len(cp)]
                     q, sc = fb.quant_act_per_token_group(dx[c], q=qs[c], scale=ss[c], stream=stream)
-                    fb.gemm_a8w8_blockscale(q, sc, wq, wsc, out=outs[c], workspace=workspace, stream=stream)
+                    fb.gemm_a8w8_blockscale(q, sc, wq, wsc, out=outs[c], workspace=workspace, stream=stream,
+                                            static_weights=True)
                     hy[c].copy_(outs[c], non_blocking=True)
         for s in range(3):
             e2e_step(s)
@@ -317,19 +319,9 @@ def run_gpu(args):
                "api": "fp8_block_scaled_a8w8_b200.quant_act_per_token_group + gemm_a8w8_blockscale (eager)"}
 
     if rank == 0:
-        detail = []
-        tot_bytes = 0.0
-        tot_ms = 0.0
-        for c, (M, N, K, *_r) in enumerate(calls):
-            by = a8w8_bytes(M, N, K)
-            fl = 2.0 * M * N * K
-            us = gemm_ms[c] * 1000.0
-            roof_us = max(by / (pk["hbm_gbs"] * 1e3), fl / (2 * pk["bf16_tflops"] * 1e6))
-            detail.append({"M": M, "N": N, "K": K, "cfg": cfgs[c], "us": round(us, 3),
-                           "GBps": round(by / us / 1e3, 1), "TFLOPS": round(fl / us / 1e6, 2),
-                           "roofline_frac": round(roof_us / us, 3)})
-            tot_bytes += by
-            tot_ms += gemm_ms[c]
+        detail = per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk)
+        tot_bytes = float(sum(a8w8_bytes(M, N, K) for (M, N, K, *_r) in calls))
+        tot_ms = gemm_ms_per_call * n_calls
         tot_flops = sum(2.0 * M * N * K for (M, N, K, *_r) in calls)
         fp8_peak = 2.0 * pk["bf16_tflops_sustained"]  # fp8 dense = 2x bf16 (nominal 4.5 / 2.25 PFLOP/s)
         hbm_bound = tot_bytes / (pk["hbm_gbs"] * 1e9) >= tot_flops / (fp8_peak * 1e12)
@@ -353,7 +345,9 @@ def run_gpu(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 -> bf16",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no dataset)",
-            "config": {"workload": args.workload, "description": inputs.WORKLOADS[args.workload], "calls_per_step": n_calls,
+            "config": {"workload": args.workload if not args.shape else "shape " + args.shape,
+                       "description": inputs.WORKLOADS[args.workload] if not args.shape else "one a8w8 call shape M,N,K",
+                       "calls_per_step": n_calls,
                        "weight_rotation_mib": ROTATE_BYTES >> 20,
                        "l2": "working set per step >> 126 MB L2 (rotated weights); no flush needed",
                        "parallelism": f"replicas x{world}", "timing": "CUDA graphs replayed, CUDA events, max over ranks"},
@@ -368,6 +362,53 @@ def run_gpu(args):
     graphs.clear()
     if world > 1:
         dist.destroy_process_group()
+
+
+def per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk, R=20, rounds=7):
+    """us/call of every distinct call shape: R back-to-back calls on rotated weight copies
+    in one CUDA graph, median over rounds interleaved across shapes ([aiter#7752] "Kernel":
+    graph replay, median of interleaved rounds)."""
+    seen, idx = set(), []
+    for c, (M, N, K, *_r) in enumerate(calls):
+        if (M, N, K) not in seen:
+            seen.add((M, N, K))
+            idx.append(c)
+    graphs = []
+    with torch.cuda.stream(stream):
+        for c in idx:
+            M, N, K, *_r = calls[c]
+            cp = wcopies[(N, K)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for r in range(R):
+                    wq, wsc = cp[r % len(cp)]
+                    fb.gemm_a8w8_blockscale(qs[c], ss[c], wq, wsc, out=outs[c], workspace=workspace, stream=stream,
+                                            static_weights=True)
+            graphs.append(g)
+    times = {c: [] for c in idx}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(rounds):
+        for c, g in zip(idx, graphs):
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+            e1.synchronize()
+            times[c].append(e0.elapsed_time(e1) * 1000.0 / R)
+    out = []
+    for c in idx:
+        M, N, K, *_r = calls[c]
+        t = sorted(times[c])
+        us = t[len(t) // 2]
+        by = a8w8_bytes(M, N, K)
+        fl = 2.0 * M * N * K
+        roof_us = max(by / (pk["hbm_gbs"] * 1e3), fl / (2 * pk["bf16_tflops"] * 1e6))
+        out.append({"M": M, "N": N, "K": K, "cfg": cfgs[c], "us": round(us, 3),
+                    "iqr_us": round(t[(3 * len(t)) // 4] - t[len(t) // 4], 3),
+                    "GBps": round(by / us / 1e3, 1), "TFLOPS": round(fl / us / 1e6, 2),
+                    "roofline_frac": round(roof_us / us, 3)})
+    del graphs
+    return out
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -452,6 +493,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="decode_sweep", choices=list(inputs.WORKLOADS))
     ap.add_argument("--impl", default="fp8bs", choices=["fp8bs", "reference"])
+    ap.add_argument("--shape", default=None, help="M,N,K: time one a8w8 call shape instead of a workload")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     args = ap.parse_args()

@@ -21,6 +21,7 @@ __all__ = [
     "gemm_bf16", "workspace_bytes", "Workspace", "dispatch_lookup", "dispatch_set_row", "dispatch_reset_table",
     "dispatch_list_configs", "dispatch_stats", "dispatch_reset_stats", "dispatch_dump_json", "dispatch_table_hash",
     "get_device_status", "status_string", "version", "OP_A8W8_BLOCKSCALE", "OP_BF16", "LIB_PATH",
+    "FLAG_STATIC_WEIGHTS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bs.so")
@@ -45,6 +46,8 @@ _PROTOS = {
     "fp8bs_quant_weight_block128": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
     "fp8bs_gemm_a8w8_blockscale": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
                                           _c_void_p, _sz, _c_void_p]),
+    "fp8bs_gemm_a8w8_blockscale_ex": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
+                                             _c_void_p, _sz, ctypes.c_uint32, _c_void_p]),
     "fp8bs_gemm_bf16": (_int, [_c_void_p, _c_void_p, _c_void_p, _int, _i64, _i64, _i64, _c_void_p, _sz, _c_void_p]),
     "fp8bs_workspace_bytes": (_sz, [_int, _i64, _i64, _i64]),
     "fp8bs_dispatch_lookup": (_int, [_int, _i64, _i64, _i64, _int, ctypes.POINTER(_i64), ctypes.POINTER(_int),
@@ -176,9 +179,16 @@ def _workspace_for(device, nbytes: int):
 
 
 # ------------------------------------------------------------------ GEMMs
+FLAG_STATIC_WEIGHTS = 1
+
+
 def gemm_a8w8_blockscale(A: torch.Tensor, a_scale: torch.Tensor, W: torch.Tensor, w_scale: torch.Tensor,
-                         out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
-    """out[M, N] bf16 = sum_g a_scale[m,g] w_scale[n/128,g] sum_{k in g} A[m,k] W[n,k] (see include/fp8bs.h)."""
+                         out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None,
+                         static_weights: bool = False):
+    """out[M, N] bf16 = sum_g a_scale[m,g] w_scale[n/128,g] sum_{k in g} A[m,k] W[n,k] (see include/fp8bs.h).
+
+    static_weights: promise that W / w_scale are not written by a kernel still running when
+    this call starts (FP8BS_FLAG_STATIC_WEIGHTS); lets the weight stream start early."""
     if not (_is_byte(A) and _is_byte(W)) or A.dim() != 2 or W.dim() != 2:
         raise ValueError("A and W must be 2-D one-byte (e4m3 code) tensors")
     M, K = A.shape
@@ -193,9 +203,14 @@ def gemm_a8w8_blockscale(A: torch.Tensor, a_scale: torch.Tensor, W: torch.Tensor
         workspace = _workspace_for(A.device, need)
     ws_ptr = _ptr(workspace) if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check("fp8bs_gemm_a8w8_blockscale",
-           lib().fp8bs_gemm_a8w8_blockscale(_ptr(A), _ptr(a_scale), _ptr(W), _ptr(w_scale), _ptr(out), M, N, K,
-                                            ws_ptr, ws_len, _stream(stream)))
+    if static_weights:
+        _check("fp8bs_gemm_a8w8_blockscale_ex",
+               lib().fp8bs_gemm_a8w8_blockscale_ex(_ptr(A), _ptr(a_scale), _ptr(W), _ptr(w_scale), _ptr(out), M, N, K,
+                                                   ws_ptr, ws_len, FLAG_STATIC_WEIGHTS, _stream(stream)))
+    else:
+        _check("fp8bs_gemm_a8w8_blockscale",
+               lib().fp8bs_gemm_a8w8_blockscale(_ptr(A), _ptr(a_scale), _ptr(W), _ptr(w_scale), _ptr(out), M, N, K,
+                                                ws_ptr, ws_len, _stream(stream)))
     return out
 
 

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "internal.h"
@@ -24,6 +25,14 @@ int device_sm_count() {
     counts[dev] = c;
   });
   return counts[dev];
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = std::getenv("FP8BS_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -47,7 +56,11 @@ static fp8bs_status check_device() {
 static fp8bs_status from_cuda(int e) { return e == 0 ? FP8BS_OK : FP8BS_ERR_CUDA; }
 
 static size_t op_workspace(int op, int64_t M, int64_t N, int64_t K, const KernelConfig& cfg) {
-  return cfg.path == kPathGemv ? gemv_workspace_bytes(op, M, N, K, cfg) : tc_workspace_bytes(op, M, N, K, cfg);
+  switch (cfg.path) {
+    case kPathGemv: return gemv_workspace_bytes(op, M, N, K, cfg);
+    case kPathGemvTma: return gemv_tma_workspace_bytes(M, N, K);
+    default: return tc_workspace_bytes(op, M, N, K, cfg);
+  }
 }
 
 }  // namespace fp8bs
@@ -105,10 +118,11 @@ static fp8bs_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int64_t kd
   return FP8BS_OK;
 }
 
-FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale(const void* A_e4m3, const float* a_scale, const void* W_e4m3,
-                                                  const float* w_scale, void* out_bf16, int64_t M, int64_t N,
-                                                  int64_t K, void* workspace, size_t workspace_bytes,
-                                                  fp8bs_stream_t stream) {
+FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const float* a_scale, const void* W_e4m3,
+                                                     const float* w_scale, void* out_bf16, int64_t M, int64_t N,
+                                                     int64_t K, void* workspace, size_t workspace_bytes, uint32_t flags,
+                                                     fp8bs_stream_t stream) {
+  if (flags & ~uint32_t(FP8BS_FLAG_STATIC_WEIGHTS)) return FP8BS_ERR_INVALID_ARG;
   if (!A_e4m3 || !a_scale || !W_e4m3 || !w_scale || !out_bf16) return FP8BS_ERR_INVALID_ARG;
   fp8bs_status st = check_gemm_shape(M, N, K, 128);
   if (st != FP8BS_OK) return st;
@@ -126,9 +140,20 @@ FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale(const void* A_e4m3, const floa
   int e;
   if (cfg->path == kPathGemv)
     e = launch_gemv_a8w8(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream);
+  else if (cfg->path == kPathGemvTma)
+    e = launch_gemv_tma_a8w8(A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace,
+                             (flags & FP8BS_FLAG_STATIC_WEIGHTS) ? 1 : 0, stream);
   else
     e = launch_tc_a8w8(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream);
   return from_cuda(e);
+}
+
+FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale(const void* A_e4m3, const float* a_scale, const void* W_e4m3,
+                                                  const float* w_scale, void* out_bf16, int64_t M, int64_t N,
+                                                  int64_t K, void* workspace, size_t workspace_bytes,
+                                                  fp8bs_stream_t stream) {
+  return fp8bs_gemm_a8w8_blockscale_ex(A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace,
+                                       workspace_bytes, 0u, stream);
 }
 
 FP8BS_API fp8bs_status fp8bs_gemm_bf16(const void* A_bf16, const void* W_bf16, void* out, int out_is_fp32, int64_t M,
@@ -157,7 +182,8 @@ FP8BS_API fp8bs_status fp8bs_gemm_bf16(const void* A_bf16, const void* W_bf16, v
 
 FP8BS_API fp8bs_status fp8bs_get_device_status(fp8bs_stream_t stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP8BS_ERR_CUDA;
-  const unsigned int v = take_device_status();
-  if (v == ~0u) return FP8BS_ERR_CUDA;
+  const unsigned int a = take_status_tc(), b = take_status_gemv_tma();
+  if (a == ~0u || b == ~0u) return FP8BS_ERR_CUDA;
+  const unsigned int v = a | b;
   return (v & kStatusTimeout) ? FP8BS_ERR_TIMEOUT : FP8BS_OK;
 }

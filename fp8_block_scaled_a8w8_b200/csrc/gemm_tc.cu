@@ -21,7 +21,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
-#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <cstring>
@@ -32,18 +31,7 @@
 
 namespace fp8bs {
 
-// Status word of the kernels in this file (bit kStatusTimeout: a bounded wait gave up).
-static __device__ unsigned int g_tc_status = 0;
-
-unsigned int take_device_status() {
-  unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_tc_status, sizeof v) != cudaSuccess) return ~0u;
-  if (v) {
-    const unsigned int zero = 0;
-    if (cudaMemcpyToSymbol(g_tc_status, &zero, sizeof zero) != cudaSuccess) return ~0u;
-  }
-  return v;
-}
+FP8BS_DEFINE_STATUS(tc)
 
 constexpr int kTcThreads = 320;
 constexpr int kBM = 128;
@@ -122,6 +110,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
   using C = TcCfg<kFp8, BN>;
   constexpr int S = C::kStages;
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* tiles = smem;
@@ -160,6 +149,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();  // the previous kernel's results are visible from here
   const uint32_t tmem_base = *tmem_slot;
 
   const int tiles_total = p.m_tiles * p.n_tiles;
@@ -177,7 +167,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
-          if (!mbar_wait_bounded(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, &g_tc_status)) {
+          if (!mbar_wait_bounded(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, &g_status)) {
             ok = false;
             break;
           }
@@ -197,7 +187,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const unsigned long long t0 = globaltimer_ns();
         while (!mbar_try_wait(full_bar(s), par))
           if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            atomicOr(&g_tc_status, kStatusTimeout);
+            atomicOr(&g_status, kStatusTimeout);
             break;
           }
       }
@@ -212,13 +202,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t d_tmem = 0;
         int tb = tile_it & 1;
         if (!kFp8) {
-          if (!mbar_wait_bounded(tempty_bar(tb), ((tile_it >> 1) & 1) ^ 1, abort_flag, &g_tc_status)) break;
+          if (!mbar_wait_bounded(tempty_bar(tb), ((tile_it >> 1) & 1) ^ 1, abort_flag, &g_status)) break;
           tc_fence_after();
           d_tmem = tmem_base + uint32_t(tb * BN);
         }
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
-          if (!mbar_wait_bounded(full_bar(s), (it / S) & 1, abort_flag, &g_tc_status)) {
+          if (!mbar_wait_bounded(full_bar(s), (it / S) & 1, abort_flag, &g_status)) {
             ok = false;
             break;
           }
@@ -226,7 +216,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           int b = 0;
           if (kFp8) {
             b = acc_it & 1;
-            if (!mbar_wait_bounded(tempty_bar(b), ((acc_it >> 1) & 1) ^ 1, abort_flag, &g_tc_status)) {
+            if (!mbar_wait_bounded(tempty_bar(b), ((acc_it >> 1) & 1) ^ 1, abort_flag, &g_status)) {
               ok = false;
               break;
             }
@@ -259,7 +249,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const unsigned long long t0 = globaltimer_ns();
         while (!mbar_try_wait(drain_bar, 0))
           if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            atomicOr(&g_tc_status, kStatusTimeout);
+            atomicOr(&g_status, kStatusTimeout);
             break;
           }
       }
@@ -293,7 +283,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const float sw = nb_ok ? __ldg(p.w_scale + int64_t(nbw) * G + kb) : 0.f;
           const float sc = sa * sw;
           const int b = acc_it & 1;
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (acc_it >> 1) & 1, abort_flag, &g_tc_status))) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (acc_it >> 1) & 1, abort_flag, &g_status))) {
             ok = false;
             break;
           }
@@ -317,7 +307,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < C::kChunks; ++c) store_row_chunk<C::kChunk>(p, row, col0 + c * C::kChunk, acc + c * C::kChunk);
       } else {
         const int b = tile_it & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (tile_it >> 1) & 1, abort_flag, &g_tc_status)))
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (tile_it >> 1) & 1, abort_flag, &g_status)))
           break;
         tc_fence_after();
         const uint32_t t_addr = lane_addr + uint32_t(b * BN + h * C::kHalfCols);
@@ -347,35 +337,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  });
-  return fn;
-}
-
-// 2-D K-major tensor map: rows of `cols` elements, box = 128 bytes x box_rows, 128-byte swizzle.
-static bool make_map(CUtensorMap* m, const void* ptr, bool fp8, int64_t rows, int64_t cols, int box_rows) {
-  auto enc = tensor_map_encoder();
-  if (!enc) return false;
-  const int esz = fp8 ? 1 : 2;
-  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
-  cuuint64_t strides[1] = {cuuint64_t(cols * esz)};
-  cuuint32_t box[2] = {cuuint32_t(kKBlockBytes / esz), cuuint32_t(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  std::memset(m, 0, sizeof(*m));
-  CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
-                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <bool kFp8, int BN>
 static int launch_tc_t(const void* A, const void* W, const TcParams& prm, void* stream) {
   using C = TcCfg<kFp8, BN>;
@@ -387,12 +348,11 @@ static int launch_tc_t(const void* A, const void* W, const TcParams& prm, void* 
   });
   if (attr_err != cudaSuccess) return int(attr_err);
   CUtensorMap ma, mb;
-  if (!make_map(&ma, A, kFp8, prm.M, prm.K, kBM) || !make_map(&mb, W, kFp8, prm.N, prm.K, BN))
+  if (!make_tma_2d_kmajor(&ma, A, kFp8, prm.M, prm.K, kBM) || !make_tma_2d_kmajor(&mb, W, kFp8, prm.N, prm.K, BN))
     return int(cudaErrorInvalidValue);
   const int tiles = prm.m_tiles * prm.n_tiles;
   const int grid = std::min(tiles, device_sm_count());
-  gemm_tc_kernel<kFp8, BN><<<grid, kTcThreads, C::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(ma, mb, prm);
-  return int(cudaGetLastError());
+  return launch_kernel(gemm_tc_kernel<kFp8, BN>, dim3(grid), dim3(kTcThreads), C::kSmemBytes, stream, ma, mb, prm);
 }
 
 size_t tc_workspace_bytes(int, int64_t, int64_t, int64_t, const KernelConfig&) { return 0; }

@@ -72,6 +72,8 @@ __device__ __forceinline__ void store_out(const GemvArgs& p, int t, int lane, co
 
 template <bool kFp8, int NB, int D>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs p) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
   const int w = blockIdx.x * kGemvWarps + (threadIdx.x >> 5);
@@ -296,8 +298,7 @@ static int launch_gemv_t(GemvArgs a, void* stream) {
   const int64_t units = int64_t(a.N / 16) * a.groups;
   a.n_active_warps = int(gemv_active_warps(units, occ));
   const int blocks = (a.n_active_warps + kGemvWarps - 1) / kGemvWarps;
-  gemv_kernel<kFp8, NB, D><<<blocks, kGemvThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
-  return int(cudaGetLastError());
+  return launch_kernel(gemv_kernel<kFp8, NB, D>, dim3(blocks), dim3(kGemvThreads), 0, stream, a);
 }
 
 template <bool kFp8, int NB>

@@ -5,6 +5,11 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <utility>
+
 #include "fp8bs.h"
 
 namespace fp8bs {
@@ -12,6 +17,7 @@ namespace fp8bs {
 enum Path : int {
   kPathGemv = 0,  // weight-streaming split-K kernel (mma.sync, small M)
   kPathTc = 1,    // tcgen05/TMEM tensor-core kernel fed by TMA
+  kPathGemvTma = 2,  // weight-streaming split-K kernel fed by TMA (mma.sync, small M)
 };
 
 // One kernel configuration a dispatch-table row can name.
@@ -35,8 +41,10 @@ const KernelConfig* dispatch(int op, int64_t M, int64_t N, int64_t K, bool recor
 // Largest M the weight-streaming path handles (8 tokens per mma.sync N block, 4 blocks).
 constexpr int64_t kGemvMaxM = 32;
 
-// Reads and clears the device-side status word (~0u on a CUDA error).
-unsigned int take_device_status();
+// Read and clear the device-side status words of the translation units whose kernels
+// wait (~0u on a CUDA error).
+unsigned int take_status_tc();
+unsigned int take_status_gemv_tma();
 
 // Device properties, cached per device.
 int device_sm_count();
@@ -51,10 +59,38 @@ int launch_gemv_a8w8(const KernelConfig& cfg, const void* A, const float* a_scal
 int launch_gemv_bf16(const KernelConfig& cfg, const void* A, const void* W, void* out, int out_fp32, int64_t M,
                      int64_t N, int64_t K, void* ws, void* stream);
 
+size_t gemv_tma_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int launch_gemv_tma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
+                         int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream);
+
+// Launch a kernel on a stream with programmatic stream serialisation (PDL) unless the
+// environment sets FP8BS_PDL=0. Returns the cudaError_t of the launch as int.
+bool pdl_enabled();
+
+// 2-D K-major TMA map, 128-byte swizzle, box = 128 bytes x box_rows.
+bool make_tma_2d_kmajor(CUtensorMap* m, const void* ptr, bool one_byte, int64_t rows, int64_t cols, int box_rows);
+
 size_t tc_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, const KernelConfig& cfg);
 int launch_tc_a8w8(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W,
                    const float* w_scale, void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream);
 int launch_tc_bf16(const KernelConfig& cfg, const void* A, const void* W, void* out, int out_fp32, int64_t M,
                    int64_t N, int64_t K, void* ws, void* stream);
+
+#ifdef __CUDACC__
+template <typename... KArgs, typename... Args>
+int launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, void* stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return int(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+}
+#endif
 
 }  // namespace fp8bs

@@ -8,9 +8,22 @@
 
 namespace fp8bs {
 
-// Device-side status word bits (the word itself lives in the translation unit of the
-// kernels that wait; fp8bs_get_device_status() reads and clears it).
+// Device-side status word (bit kStatusTimeout: a bounded wait gave up). Without
+// relocatable device code a __device__ variable cannot be shared between translation
+// units, so every .cu file that waits has its own word (FP8BS_DEFINE_STATUS) and a host
+// accessor that reads and clears it; fp8bs_get_device_status() ORs them.
 constexpr unsigned int kStatusTimeout = 1u;
+#define FP8BS_DEFINE_STATUS(tu)                                                    \
+  static __device__ unsigned int g_status = 0;                                      \
+  unsigned int take_status_##tu() {                                                 \
+    unsigned int v = 0;                                                             \
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof v) != cudaSuccess) return ~0u;    \
+    if (v) {                                                                        \
+      const unsigned int zero = 0;                                                  \
+      if (cudaMemcpyToSymbol(g_status, &zero, sizeof zero) != cudaSuccess) return ~0u; \
+    }                                                                               \
+    return v;                                                                       \
+  }
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
@@ -23,6 +36,14 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// Every kernel lets the next kernel in the stream launch as soon as all of its CTAs are
+// running (pdl_trigger), and waits for the previous kernel to complete and flush its
+// memory (pdl_wait) before its first global-memory access. Without the launch attribute
+// both are no-ops, so the kernels are correct either way.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -172,6 +193,16 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------- gpu-scope atomics
+// fetch-add with acquire-release semantics at gpu scope: after a CTA barrier, one
+// thread's release publishes every CTA thread's earlier stores (cumulativity), and its
+// acquire makes the other contributors' stores visible to the CTA after the next barrier.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 // ---------------------------------------------------------------- global loads

@@ -29,6 +29,8 @@ __device__ __forceinline__ uint32_t cvt4_e4m3(float a, float b, float c, float d
 __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
                                                         int64_t ld_x, uint8_t* __restrict__ q,
                                                         float* __restrict__ scale) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t G = K / 128;
   const int64_t total = M * G;
   const int lane = threadIdx.x & 31;
@@ -64,6 +66,8 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
 // One CTA (256 threads) per 128x128 block; thread t owns row t/2, 64 columns.
 __global__ void __launch_bounds__(256) quant_weight_kernel(const float* __restrict__ w, int64_t N, int64_t K,
                                                            uint8_t* __restrict__ q, float* __restrict__ scale) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t G = K / 128;
   const int64_t nb = blockIdx.y;
   const int64_t g = blockIdx.x;
@@ -103,15 +107,13 @@ int launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q,
   const int64_t need = (groups + 15) / 16;  // 16 groups per 256-thread block per pass
   const int64_t cap = int64_t(device_sm_count()) * 8;
   const int blocks = int(need < cap ? need : cap);
-  quant_act_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(x), M, K, ld_x, static_cast<uint8_t*>(q), scale);
-  return int(cudaGetLastError());
+  return launch_kernel(quant_act_kernel, dim3(blocks), dim3(256), 0, stream, static_cast<const uint16_t*>(x), M, K,
+                       ld_x, static_cast<uint8_t*>(q), scale);
 }
 
 int launch_quant_weight(const float* w, int64_t N, int64_t K, void* q, float* scale, void* stream) {
   dim3 grid(unsigned(K / 128), unsigned((N + 127) / 128));
-  quant_weight_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(w, N, K, static_cast<uint8_t*>(q), scale);
-  return int(cudaGetLastError());
+  return launch_kernel(quant_weight_kernel, grid, dim3(256), 0, stream, w, N, K, static_cast<uint8_t*>(q), scale);
 }
 
 }  // namespace fp8bs

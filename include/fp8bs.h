@@ -107,6 +107,23 @@ fp8bs_status fp8bs_gemm_a8w8_blockscale(const void* A_e4m3, const float* a_scale
                                         int64_t K, void* workspace, size_t workspace_bytes,
                                         fp8bs_stream_t stream);
 
+/* Flags for fp8bs_gemm_a8w8_blockscale_ex. */
+enum {
+  /* W_e4m3 and w_scale are not written by any kernel that can still be running when this
+   * call's kernel starts (true of inference weights loaded once). The weight-streaming
+   * kernel then starts fetching W before the preceding kernel in the stream has finished
+   * (programmatic dependent launch), overlapping its weight stream with that kernel's
+   * tail; activations, scales and the workspace are still read only after it finished. */
+  FP8BS_FLAG_STATIC_WEIGHTS = 1u
+};
+
+/* fp8bs_gemm_a8w8_blockscale with flags (a bitwise OR of FP8BS_FLAG_*; unknown bits give
+ * FP8BS_ERR_INVALID_ARG). fp8bs_gemm_a8w8_blockscale is this call with flags = 0. */
+fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const float* a_scale, const void* W_e4m3,
+                                           const float* w_scale, void* out_bf16, int64_t M, int64_t N,
+                                           int64_t K, void* workspace, size_t workspace_bytes, uint32_t flags,
+                                           fp8bs_stream_t stream);
+
 /*
  * Companion bf16 GEMM for the small-N router / indexer projections ([cookbook#8]:
  * the live BF16 lookups are the MoE router and the DSA indexer's weights_proj;

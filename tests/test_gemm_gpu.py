@@ -51,10 +51,17 @@ def test_gemv_path_parity(M, N, K):
     check_a8w8(_run(*case), *case)
 
 
-@pytest.mark.parametrize("cfg", ["a8w8_gemv_d2", "a8w8_gemv_d3", "a8w8_gemv_d4"])
+@pytest.mark.parametrize("cfg", ["a8w8_gemv_d2", "a8w8_gemv_d3", "a8w8_gemv_d4", "a8w8_gemv_tma"])
 @pytest.mark.parametrize("M", [1, 7, 16, 25])
 def test_gemv_depths(cfg, M):
     case = _raw_case(M, 400, 1408, seed=M + 77)
+    check_a8w8(_run(*case, cfg=cfg), *case)
+
+
+@pytest.mark.parametrize("cfg", ["a8w8_gemv_d4", "a8w8_gemv_tma"])
+@pytest.mark.parametrize("M,N,K", [(1, 16, 128), (5, 144, 128), (32, 34816, 5120), (12, 5120, 6144), (2, 130 * 16, 3968)])
+def test_gemv_kernels_shapes(cfg, M, N, K):
+    case = _raw_case(M, N, K, seed=M + N + K)
     check_a8w8(_run(*case, cfg=cfg), *case)
 
 
@@ -178,3 +185,37 @@ def test_workspace_left_zero_and_shared_across_shapes():
         torch.cuda.synchronize()
         assert int(ws.count_nonzero()) == 0
         check_a8w8(y, *case)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 5120, 6144), (16, 34816, 5120), (9, 2048, 1024), (3, 144, 384)])
+def test_static_weights_flag_bit_identical(M, N, K):
+    """FP8BS_FLAG_STATIC_WEIGHTS only moves the weight fetch earlier: same bits, also when
+    the call follows a kernel that writes its activations (the quantiser) in one graph."""
+    case = _raw_case(M, N, K, seed=7 + M)
+    A, a_s, W, w_s = (codes_to_device(case[0]), torch.from_numpy(case[1]).cuda(), codes_to_device(case[2]),
+                      torch.from_numpy(case[3]).cuda())
+    ref = fb.gemm_a8w8_blockscale(A, a_s, W, w_s)
+    y = fb.gemm_a8w8_blockscale(A, a_s, W, w_s, static_weights=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits(y), bf16_bits(ref))
+    # quantiser -> GEMM chains in one graph, the GEMM reading what the quantiser wrote
+    x = inputs.activation_bf16(M, K, seed=M)
+    xd = x.cuda()
+    q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device="cuda")
+    s = torch.empty((M, K // 128), dtype=torch.float32, device="cuda")
+    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(max(fb.workspace_bytes(OP, M, N, K), 256), dtype=torch.uint8, device="cuda")
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        for _ in range(3):
+            fb.quant_act_per_token_group(xd, q=q, scale=s, stream=st)
+            fb.gemm_a8w8_blockscale(q, s, W, w_s, out=out, workspace=ws, stream=st, static_weights=True)
+    g.replay()
+    torch.cuda.synchronize()
+    q2, s2 = fb.quant_act_per_token_group(xd)
+    ref2 = fb.gemm_a8w8_blockscale(q2, s2, W, w_s)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits(out), bf16_bits(ref2))
+    assert int(ws.count_nonzero()) == 0
