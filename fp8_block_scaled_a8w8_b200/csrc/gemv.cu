@@ -280,8 +280,6 @@ static int gemv_occ(int nb, int depth) {
   }
 }
 
-static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
 size_t gemv_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, const KernelConfig& cfg) {
   const bool fp8 = op == FP8BS_OP_A8W8_BLOCKSCALE;
   const int nb = gemv_nb(M);
@@ -289,7 +287,7 @@ size_t gemv_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, const Kerne
   const int64_t units = (N / 16) * groups;
   const int occ = fp8 ? gemv_occ<true>(nb, cfg.gemv_depth) : gemv_occ<false>(nb, cfg.gemv_depth);
   const int64_t warps = gemv_active_warps(units, occ);
-  return align256(size_t(N / 16) * sizeof(unsigned)) + size_t(2 * warps) * nb * 4 * 32 * sizeof(float);
+  return kCounterBytes + size_t(2 * warps) * nb * 4 * 32 * sizeof(float);
 }
 
 template <bool kFp8, int NB, int D>
@@ -312,6 +310,7 @@ static int launch_gemv_depth(const KernelConfig& cfg, const GemvArgs& a, void* s
 
 template <bool kFp8>
 static int launch_gemv_nb(const KernelConfig& cfg, const GemvArgs& a, void* stream) {
+  if (a.N / 16 > kMaxCounters) return int(cudaErrorInvalidValue);
   switch (gemv_nb(a.M)) {
     case 1: return launch_gemv_depth<kFp8, 1>(cfg, a, stream);
     case 2: return launch_gemv_depth<kFp8, 2>(cfg, a, stream);
@@ -335,7 +334,7 @@ static GemvArgs make_args(const void* A, const float* a_scale, const void* W, co
   a.row_bytes = int(fp8 ? K : 2 * K);
   a.groups = int(fp8 ? K / 128 : K / 64);
   a.counter = static_cast<unsigned*>(ws);
-  a.part = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(size_t(N / 16) * sizeof(unsigned)));
+  a.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
   a.out_fp32 = out_fp32;
   return a;
 }

@@ -21,8 +21,9 @@
 // any shape. A block covered by one CTA is written directly; a block shared by several
 // CTAs is finished by the last to arrive (atomic counter per block), which sums the
 // float32 partials in CTA order -- fixed, so results are bit-reproducible -- writes the
-// bf16 output, and zeroes the partials and the counter (the workspace is left
-// zero-filled). A CTA leaves partial sums for at most two blocks (the first and last of
+// bf16 output and resets the block's counter to zero. Partial sums are always
+// overwritten before their counter is incremented, so they need no clearing; the
+// counters live in a fixed region at the start of the workspace and are left at zero. A CTA leaves partial sums for at most two blocks (the first and last of
 // its range); both are plain stores while streaming, published together at the end of
 // the range by one acq_rel atomic per block after a CTA barrier, so nothing stalls the
 // stream mid-range.
@@ -91,6 +92,47 @@ __device__ __forceinline__ void gt_store(const GtParams& p, int b, int w, int la
       const int token = nb * 8 + 2 * tig + (i & 1);
       if (token < p.M) p.out[int64_t(token) * p.N + n0 + (i >= 2 ? 8 : 0)] = __float2bfloat16_rn(v[nb][i]);
     }
+}
+
+// Finish block b if this CTA was its last contributor (arrival count old == contributors - 1):
+// sum the contributors' partials in CTA order (a fixed order: bit-reproducible results),
+// four loads in flight at a time, store the output, reset the block's counter.
+// Contributor cc > cf of block b started its range inside b (its slot 0); the first
+// contributor cf used slot 0 only if its range started exactly at b's first unit, else b
+// was its last block (slot 1).
+template <int NB>
+__device__ __forceinline__ void gt_finish_block(const GtParams& p, int b, unsigned old, int64_t U, int64_t Cn,
+                                                int64_t G, int w, int lane) {
+  const int64_t cf = cta_of_unit(int64_t(b) * G, U, Cn);
+  const int64_t cl = cta_of_unit(int64_t(b + 1) * G - 1, U, Cn);
+  if (old != unsigned(cl - cf)) return;
+  const int cf_slot = (U * cf / Cn >= int64_t(b) * G) ? 0 : 1;
+  float sum[NB][4];
+#pragma unroll
+  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sum[nb][i] = 0.f;
+  for (int64_t c0 = cf; c0 <= cl; c0 += 4) {
+    float v[4][NB][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t cc = c0 + j;
+      const int64_t sl = 2 * cc + (cc == cf ? cf_slot : 0);
+      const float* src = p.part + (sl * kGtConsumers + w) * (NB * 4 * 32);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[j][nb][i] = cc <= cl ? __ldcg(src + (nb * 4 + i) * 32 + lane) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sum[nb][i] += v[j][nb][i];
+  }
+  gt_store<NB>(p, b, w, lane, sum);
+  if (w == 0 && lane == 0) p.counter[b] = 0u;
 }
 
 template <int NB>
@@ -206,7 +248,7 @@ __global__ void __launch_bounds__(kGtThreads, 1)
       off_w[c] = uint32_t((16 * w + gid) * 128) + chunk;
       off_a[c] = uint32_t(C::kWBytes + gid * 128) + chunk;
     }
-    int pending[2] = {-1, -1};  // blocks this CTA left partial sums for (at most its first and last)
+    int pend0 = -1, pend1 = -1;  // blocks this CTA left partial sums for (at most its first and last)
     int n_pending = 0;
     int it = 0;
     bool aborted = false;
@@ -275,7 +317,11 @@ __global__ void __launch_bounds__(kGtThreads, 1)
           for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
             for (int i = 0; i < 4; ++i) __stcg(dst + (nb * 4 + i) * 32 + lane, acc[nb][i]);
-          if (n_pending < 2) pending[n_pending++] = b;
+          if (n_pending == 0)
+            pend0 = b;
+          else
+            pend1 = b;
+          ++n_pending;
         }
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
@@ -289,82 +335,20 @@ __global__ void __launch_bounds__(kGtThreads, 1)
     }
     // ---- publish the partial sums; the last contributor of a block reduces it
     consumer_bar();  // every consumer thread's partial stores happen before the release below
-    if (w == 0 && lane < n_pending) red_slot[lane] = aborted ? 0u : atom_add_acq_rel_gpu(p.counter + pending[lane], 1u);
-    consumer_bar();
-    // blocks this CTA finishes (it was the last contributor)
-    int rb[2] = {-1, -1};
-    int64_t rcf[2] = {0, 0}, rn[2] = {0, 0};
-    int nr = 0;
-    for (int k = 0; k < n_pending && !aborted; ++k) {
-      const int pb = pending[k];
-      const int64_t cf = cta_of_unit(int64_t(pb) * G, U, Cn);
-      const int64_t cl = cta_of_unit(int64_t(pb + 1) * G - 1, U, Cn);
-      if (red_slot[k] != unsigned(cl - cf)) continue;
-      rb[nr] = pb;
-      rcf[nr] = cf;
-      rn[nr] = cl - cf + 1;
-      ++nr;
+    if (w == 0 && lane < n_pending) {
+      const int pb = lane == 0 ? pend0 : pend1;
+      red_slot[lane] = aborted ? 0u : atom_add_acq_rel_gpu(p.counter + pb, 1u);
     }
-    if (nr > 0) {
-      // every contributor's partial (of both blocks) is loaded before any is added, so the
-      // L2 round trips overlap; each block's partials are then summed in CTA order -- a
-      // fixed order, so results are bit-reproducible
-      constexpr int kChunk = NB <= 2 ? 8 : 4;
-      float sum0[NB][4], sum1[NB][4];
-#pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sum0[nb][i] = sum1[nb][i] = 0.f;
-      const int64_t total = rn[0] + rn[1];
-      for (int64_t j0 = 0; j0 < total; j0 += kChunk) {
-        float v[kChunk][NB][4];
-        float* src[kChunk];
-#pragma unroll
-        for (int jj = 0; jj < kChunk; ++jj) {
-          const int64_t j = j0 + jj;
-          src[jj] = nullptr;
-          if (j >= total) break;
-          const int k = j < rn[0] ? 0 : 1;
-          const int64_t cc = rcf[k] + (k == 0 ? j : j - rn[0]);
-          const int fb = int((U * cc / Cn) / G);
-          const int sl = 2 * int(cc) + (rb[k] == fb ? 0 : 1);
-          src[jj] = p.part + (int64_t(sl) * kGtConsumers + w) * (NB * 4 * 32);
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) v[jj][nb][i] = __ldcg(src[jj] + (nb * 4 + i) * 32 + lane);
-        }
-#pragma unroll
-        for (int jj = 0; jj < kChunk; ++jj) {
-          const int64_t j = j0 + jj;
-          if (j >= total) break;
-          const bool first = j < rn[0];
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              if (first)
-                sum0[nb][i] += v[jj][nb][i];
-              else
-                sum1[nb][i] += v[jj][nb][i];
-              __stcg(src[jj] + (nb * 4 + i) * 32 + lane, 0.f);  // leave the workspace zero-filled
-            }
-        }
-      }
-      gt_store<NB>(p, rb[0], w, lane, sum0);
-      if (nr > 1) gt_store<NB>(p, rb[1], w, lane, sum1);
-      if (w == 0 && lane == 0) {
-        p.counter[rb[0]] = 0u;
-        if (nr > 1) p.counter[rb[1]] = 0u;
-      }
+    consumer_bar();
+    if (!aborted) {
+      if (n_pending > 0) gt_finish_block<NB>(p, pend0, red_slot[0], U, Cn, G, w, lane);
+      if (n_pending > 1) gt_finish_block<NB>(p, pend1, red_slot[1], U, Cn, G, w, lane);
     }
   }
   __syncthreads();
 }
 
 // ---------------------------------------------------------------- host side
-static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-
 static int gt_ctas(int64_t M, int64_t N, int64_t K) {
   (void)M;
   const int64_t units = ((N + kGtRows - 1) / kGtRows) * (K / 128);
@@ -373,15 +357,14 @@ static int gt_ctas(int64_t M, int64_t N, int64_t K) {
 
 size_t gemv_tma_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   const int nb = int((M + 7) / 8);
-  const int64_t nblk = (N + kGtRows - 1) / kGtRows;
-  return align256(size_t(nblk) * sizeof(unsigned)) +
-         size_t(2) * gt_ctas(M, N, K) * kGtConsumers * nb * 4 * 32 * sizeof(float);
+  return kCounterBytes + size_t(2) * gt_ctas(M, N, K) * kGtConsumers * nb * 4 * 32 * sizeof(float);
 }
 
 template <int NB>
 static int launch_gt(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out, int64_t M,
                      int64_t N, int64_t K, void* ws, int static_w, void* stream) {
   using Cc = GtCfg<NB>;
+  if ((N + kGtRows - 1) / kGtRows > kMaxCounters) return int(cudaErrorInvalidValue);
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
@@ -402,7 +385,7 @@ static int launch_gt(const void* A, const float* a_scale, const void* W, const f
   p.n_ctas = gt_ctas(M, N, K);
   p.static_w = static_w;
   p.counter = static_cast<unsigned*>(ws);
-  p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(size_t(p.nblk) * sizeof(unsigned)));
+  p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
   return launch_kernel(gemv_tma_kernel<NB>, dim3(p.n_ctas), dim3(kGtThreads), Cc::kSmemBytes, stream, mw, ma, p);
 }
 

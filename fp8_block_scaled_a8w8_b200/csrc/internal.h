@@ -38,6 +38,13 @@ const KernelConfig* default_config(int op, int64_t M, int64_t N, int64_t K);
 // Table lookup with the padded-M walk; record != 0 counts it in the census.
 const KernelConfig* dispatch(int op, int64_t M, int64_t N, int64_t K, bool record, int64_t* padded_M, bool* hit);
 
+// Workspace layout shared by the split-K kernels: a fixed region of arrival counters
+// (one per output block, at most kMaxCounters) followed by the partial sums. The counter
+// region does not depend on the shape, so one call's counters never land on another
+// call's partial sums; every call leaves its counters at zero.
+constexpr int64_t kMaxCounters = 65536;
+constexpr size_t kCounterBytes = size_t(kMaxCounters) * 4;
+
 // Largest M the weight-streaming path handles (8 tokens per mma.sync N block, 4 blocks).
 constexpr int64_t kGemvMaxM = 32;
 

@@ -93,9 +93,11 @@ fp8bs_status fp8bs_quant_weight_block128(const float* w_f32, int64_t N, int64_t 
  * out_bf16 [M,N]: device pointers. Requires M,N,K > 0, K % 128 == 0, N % 16 == 0.
  * workspace: device scratch of at least fp8bs_workspace_bytes(FP8BS_OP_A8W8_BLOCKSCALE, M, N, K)
  * bytes (may be NULL when that is 0). It must be zero-filled once before its first
- * use; every call leaves it zero-filled again (it holds split-K partial sums and
- * self-resetting arrival counters), so one workspace serves any number of calls on
- * one stream. Calls that may run concurrently need separate workspaces.
+ * use. It holds split-K arrival counters, which every call leaves at zero, and partial
+ * sums, whose contents between calls are unspecified; so one workspace serves any
+ * number of calls of any shapes issued in order on one stream. Calls that may run
+ * concurrently need separate workspaces. After a call reported FP8BS_ERR_TIMEOUT
+ * (fp8bs_get_device_status) the workspace must be zero-filled again.
  * The kernel is picked by the dispatch table (fp8bs_dispatch_lookup): a
  * weight-streaming split-K kernel for small M, a tcgen05/TMEM tensor-core kernel
  * fed by TMA otherwise. Results are deterministic (split-K partial sums are
