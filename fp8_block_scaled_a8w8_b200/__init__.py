@@ -21,7 +21,7 @@ __all__ = [
     "gemm_bf16", "workspace_bytes", "Workspace", "dispatch_lookup", "dispatch_set_row", "dispatch_reset_table",
     "dispatch_list_configs", "dispatch_stats", "dispatch_reset_stats", "dispatch_dump_json", "dispatch_table_hash",
     "get_device_status", "status_string", "version", "OP_A8W8_BLOCKSCALE", "OP_BF16", "LIB_PATH",
-    "FLAG_STATIC_WEIGHTS",
+    "FLAG_STATIC_WEIGHTS", "gemm_a8w8_blockscale_noalloc",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bs.so")
@@ -48,6 +48,8 @@ _PROTOS = {
                                           _c_void_p, _sz, _c_void_p]),
     "fp8bs_gemm_a8w8_blockscale_ex": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
                                              _c_void_p, _sz, ctypes.c_uint32, _c_void_p]),
+    "fp8bs_gemm_a8w8_blockscale_noalloc": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64,
+                                                  _i64, _c_void_p]),
     "fp8bs_gemm_bf16": (_int, [_c_void_p, _c_void_p, _c_void_p, _int, _i64, _i64, _i64, _c_void_p, _sz, _c_void_p]),
     "fp8bs_workspace_bytes": (_sz, [_int, _i64, _i64, _i64]),
     "fp8bs_dispatch_lookup": (_int, [_int, _i64, _i64, _i64, _int, ctypes.POINTER(_i64), ctypes.POINTER(_int),
@@ -211,6 +213,21 @@ def gemm_a8w8_blockscale(A: torch.Tensor, a_scale: torch.Tensor, W: torch.Tensor
         _check("fp8bs_gemm_a8w8_blockscale",
                lib().fp8bs_gemm_a8w8_blockscale(_ptr(A), _ptr(a_scale), _ptr(W), _ptr(w_scale), _ptr(out), M, N, K,
                                                 ws_ptr, ws_len, _stream(stream)))
+    return out
+
+
+def gemm_a8w8_blockscale_noalloc(A: torch.Tensor, a_scale: torch.Tensor, W: torch.Tensor, w_scale: torch.Tensor,
+                                 out: torch.Tensor | None = None, stream=None):
+    """gemm_a8w8_blockscale for M <= 32 without a workspace: for callers that cannot allocate
+    device memory when they issue the GEMM (see include/fp8bs.h). Its scratch is one array in
+    the library image shared by all calls, so calls must not overlap on the GPU."""
+    M, K = A.shape
+    N = W.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    _check("fp8bs_gemm_a8w8_blockscale_noalloc",
+           lib().fp8bs_gemm_a8w8_blockscale_noalloc(_ptr(A), _ptr(a_scale), _ptr(W), _ptr(w_scale), _ptr(out), M, N,
+                                                    K, _stream(stream)))
     return out
 
 

@@ -156,6 +156,22 @@ FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale(const void* A_e4m3, const floa
                                        workspace_bytes, 0u, stream);
 }
 
+FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale_noalloc(const void* A_e4m3, const float* a_scale,
+                                                          const void* W_e4m3, const float* w_scale, void* out_bf16,
+                                                          int64_t M, int64_t N, int64_t K, fp8bs_stream_t stream) {
+  if (!A_e4m3 || !a_scale || !W_e4m3 || !w_scale || !out_bf16) return FP8BS_ERR_INVALID_ARG;
+  fp8bs_status st = check_gemm_shape(M, N, K, 128);
+  if (st != FP8BS_OK) return st;
+  if (!aligned16(A_e4m3) || !aligned16(W_e4m3) || !aligned16(out_bf16) || !aligned16(a_scale) || !aligned16(w_scale))
+    return FP8BS_ERR_ALIGNMENT;
+  st = check_device();
+  if (st != FP8BS_OK) return st;
+  int too_big = 0;
+  const int e = launch_gemv_tma_noalloc(A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, stream, &too_big);
+  if (too_big) return FP8BS_ERR_UNSUPPORTED;
+  return from_cuda(e);
+}
+
 FP8BS_API fp8bs_status fp8bs_gemm_bf16(const void* A_bf16, const void* W_bf16, void* out, int out_is_fp32, int64_t M,
                                        int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                                        fp8bs_stream_t stream) {

@@ -400,4 +400,49 @@ int launch_gemv_tma_a8w8(const void* A, const float* a_scale, const void* W, con
   }
 }
 
+// ---------------------------------------------------------------- allocation-free variant
+// Some callers cannot allocate device memory at the point where they issue a GEMM: code
+// running under an allocator that is frozen or owned by someone else (a serving engine
+// whose memory pool was sized once at start-up, a plugin inside a host framework, code
+// that must not trigger an allocation-induced synchronisation), or code with no handle on
+// an allocator at all. For them the weight-streaming kernel can take its split-K scratch
+// from a fixed array that is part of the loaded library image instead of a caller-owned
+// workspace. Every GPU that loads the library holds this array until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB: counters + partial sums
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array on the current device (looked up once per device;
+// the array's host-side name is not a device address). nullptr if the lookup failed.
+static void* noalloc_scratch_ptr() {
+  static void* ptrs[64];
+  static cudaError_t errs[64];
+  static std::once_flag once[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::call_once(once[dev], [dev] {
+    void* p = nullptr;
+    errs[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    ptrs[dev] = errs[dev] == cudaSuccess ? p : nullptr;
+  });
+  return ptrs[dev];
+}
+
+int launch_gemv_tma_noalloc(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
+                            int64_t M, int64_t N, int64_t K, void* stream, int* too_big) {
+  *too_big = 0;
+  if (M > kGemvMaxM || gemv_tma_workspace_bytes(M, N, K) > kNoAllocScratchBytes ||
+      (N + kGtRows - 1) / kGtRows > kMaxCounters) {
+    *too_big = 1;
+    return int(cudaErrorInvalidValue);
+  }
+  void* scratch = noalloc_scratch_ptr();
+  if (!scratch) return int(cudaErrorInvalidSymbol);
+  // The array keeps whatever the previous call left in it; the arrival counters this call
+  // uses must start at zero, so clear them (partial sums are always written before read).
+  const size_t counter_bytes = size_t((N + kGtRows - 1) / kGtRows) * sizeof(unsigned);
+  cudaError_t e = cudaMemsetAsync(scratch, 0, counter_bytes, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return int(e);
+  return launch_gemv_tma_a8w8(A, a_scale, W, w_scale, out, M, N, K, scratch, 0, stream);
+}
+
 }  // namespace fp8bs

@@ -74,6 +74,11 @@ int launch_gemv_tma_a8w8(const void* A, const float* a_scale, const void* W, con
 // environment sets FP8BS_PDL=0. Returns the cudaError_t of the launch as int.
 bool pdl_enabled();
 
+// Allocation-free variant of the weight-streaming kernel: its scratch is a fixed array in
+// the library image. *too_big = 1 when the shape needs more scratch than the array holds.
+int launch_gemv_tma_noalloc(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
+                            int64_t M, int64_t N, int64_t K, void* stream, int* too_big);
+
 // 2-D K-major TMA map, 128-byte swizzle, box = 128 bytes x box_rows.
 bool make_tma_2d_kmajor(CUtensorMap* m, const void* ptr, bool one_byte, int64_t rows, int64_t cols, int box_rows);
 

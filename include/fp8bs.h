@@ -127,6 +127,30 @@ fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const float* a_sc
                                            fp8bs_stream_t stream);
 
 /*
+ * The a8w8 block-scaled GEMM for decode-sized M without any caller-provided memory.
+ * (No counterpart in the pages: an addition for callers that cannot allocate.)
+ * Some callers cannot allocate device memory where they issue a GEMM -- their memory pool
+ * is fixed or owned by a host framework, or an allocation there would synchronise -- so
+ * they cannot supply the workspace fp8bs_gemm_a8w8_blockscale needs. This entry point
+ * runs the same weight-streaming split-K kernel with its scratch taken from one fixed
+ * 8 MiB array that is part of the library image (every GPU that loads the library holds
+ * it until the process exits); it calls no allocator of any kind.
+ * Arguments and result as fp8bs_gemm_a8w8_blockscale, without the workspace.
+ * Limits: M <= 32 and shapes whose split-K scratch fits the array (on a 148-SM B200 every
+ * N up to 65536 * 128 rows qualifies); other shapes return FP8BS_ERR_UNSUPPORTED and
+ * launch nothing.
+ * The first call on a device looks up the array's device address (once per device, with
+ * that device current); make that first call before any CUDA stream capture.
+ * Every call uses the same array and it keeps the last call's contents: each call clears
+ * the arrival counters it uses (an asynchronous memset on the stream) before its kernel.
+ * Calls that can overlap on the GPU (different streams, or concurrent host threads) race
+ * on the array and give wrong results; issue them in order on one stream.
+ */
+fp8bs_status fp8bs_gemm_a8w8_blockscale_noalloc(const void* A_e4m3, const float* a_scale, const void* W_e4m3,
+                                                const float* w_scale, void* out_bf16, int64_t M, int64_t N,
+                                                int64_t K, fp8bs_stream_t stream);
+
+/*
  * Companion bf16 GEMM for the small-N router / indexer projections ([cookbook#8]:
  * the live BF16 lookups are the MoE router and the DSA indexer's weights_proj;
  * [aiter#7247] "Technical Details": N = 32..1024, some with fp32 output).
