@@ -52,6 +52,24 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def measured_traffic(kernel_key, algorithmic_bytes_per_launch):
+    """DRAM bytes per launch from the committed ncu capture (profiles/traffic.json), scaled
+    from the captured shape to this workload by algorithmic bytes (the kernels stream their
+    operands once, so traffic grows in proportion). None if the kernel source changed since
+    the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel_key)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != d["sha256_16"]:
+        return None
+    return round(d["dram_bytes"] / d["algorithmic_bytes"] * algorithmic_bytes_per_launch)
+
+
 def a8w8_bytes(M, N, K):
     """Algorithmic bytes of one call: A + a_scale + W + w_scale + out."""
     G = K // 128
@@ -319,7 +337,8 @@ def run_gpu(args):
                "api": "fp8_block_scaled_a8w8_b200.quant_act_per_token_group + gemm_a8w8_blockscale (eager)"}
 
     if rank == 0:
-        detail = per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk)
+        detail = per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk) \
+            if args.detail else None
         tot_bytes = float(sum(a8w8_bytes(M, N, K) for (M, N, K, *_r) in calls))
         tot_ms = gemm_ms_per_call * n_calls
         tot_flops = sum(2.0 * M * N * K for (M, N, K, *_r) in calls)
@@ -335,7 +354,10 @@ def run_gpu(args):
             roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                     "frac": round(achieved / fp8_peak, 4),
                     "peak_source": f"2 x {pk['source']} sustained bf16 cuBLAS (fp8/bf16 nominal ratio 2)"}
-        roof["traffic"] = None
+        key = "gemv_tma" if all(c == "a8w8_gemv_tma" for c in cfgs) else \
+            "gemm_tc" if all(c.startswith("a8w8_tc") for c in cfgs) else None
+        roof["traffic"] = measured_traffic(key, tot_bytes / n_calls) if key else None
+        roof["traffic_note"] = "DRAM bytes per launch (average call), ncu capture in profiles/ scaled by algorithmic bytes"
         roof["kernel"] = "gemm_a8w8_blockscale: " + ", ".join(sorted(set(cfgs)))
         roof["algorithmic_bytes_per_step"] = int(tot_bytes)
         roof["gemm_us_per_step"] = round(tot_ms * 1000.0, 2)
@@ -496,6 +518,8 @@ def main():
     ap.add_argument("--shape", default=None, help="M,N,K: time one a8w8 call shape instead of a workload")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-detail", dest="detail", action="store_false",
+                    help="skip the per-shape back-to-back timing table (for profiler runs)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
