@@ -13,6 +13,7 @@ from __future__ import annotations
 import argparse
 import concurrent.futures as cf
 import os
+import re
 import subprocess
 import sys
 
@@ -35,6 +36,32 @@ def _headers():
     return hs
 
 
+# Kernels that move registers between warpgroups with setmaxnreg: the split is only valid if
+# ptxas gives every thread exactly this many registers at launch (otherwise setmaxnreg.inc
+# would wait for registers that do not exist), so the build checks it.
+REGISTER_CONTRACTS = {"gemm_tc.cu": ("gemm_tc_kernel", 168)}
+
+
+def _check_register_contract(src: str, log: str) -> None:
+    if src not in REGISTER_CONTRACTS:
+        return
+    needle, regs = REGISTER_CONTRACTS[src]
+    lines = log.splitlines()
+    seen = 0
+    for i, line in enumerate(lines):
+        if "Compiling entry function" in line and needle in line:
+            for nxt in lines[i + 1:i + 6]:
+                m = re.search(r"Used (\d+) registers", nxt)
+                if m:
+                    seen += 1
+                    if int(m.group(1)) != regs:
+                        raise RuntimeError(f"{src}: {line.strip()} uses {m.group(1)} registers, the setmaxnreg split "
+                                           f"needs exactly {regs}")
+                    break
+    if seen == 0:
+        raise RuntimeError(f"{src}: no ptxas register report for {needle}")
+
+
 def _compile(src: str, force: bool, ptxas_verbose: bool) -> tuple[str, str]:
     path = os.path.join(CSRC, src)
     obj = os.path.join(BUILD, src + ".o")
@@ -44,12 +71,17 @@ def _compile(src: str, force: bool, ptxas_verbose: bool) -> tuple[str, str]:
     cmd = [NVCC, *ARCH, *COMMON, "-c", path, "-o", obj]
     if src.endswith(".cpp"):
         cmd[1:1] = ["-x", "cu"]
-    if ptxas_verbose and src.endswith(".cu"):
+    if (ptxas_verbose and src.endswith(".cu")) or src in REGISTER_CONTRACTS:
         cmd.append("-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
-    return obj, r.stderr
+    try:
+        _check_register_contract(src, r.stderr)
+    except RuntimeError:
+        os.remove(obj)
+        raise
+    return obj, r.stderr if ptxas_verbose else ""
 
 
 def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) -> str:

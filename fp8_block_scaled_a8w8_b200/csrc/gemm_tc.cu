@@ -3,7 +3,7 @@
 //
 //   warp 0        TMA producer: one 128-row A box and one BN-row W box per K block
 //   warp 1        TMEM allocator and MMA issuer (one elected thread)
-//   warps 2..9    epilogue: TMEM -> registers -> bf16/f32 -> global
+//   warps 4..11   epilogue: TMEM -> registers -> bf16/f32 -> global
 //
 // a8w8 block scale: a 128-wide K group is one K block. Each group's four
 // tcgen05.mma (K = 32 each) write a fresh float32 partial P_g into one of two TMEM
@@ -33,7 +33,16 @@ namespace fp8bs {
 
 FP8BS_DEFINE_STATUS(tc)
 
-constexpr int kTcThreads = 320;
+// 12 warps = 3 warpgroups. Warpgroup 0: warp 0 TMA producer, warp 1 TMEM allocator and MMA
+// issuer, warps 2-3 idle. Warpgroups 1-2 (warps 4-11): epilogue. Registers are moved from
+// warpgroup 0 to the epilogue with setmaxnreg: the launch gives every thread kLaunchRegs
+// (checked by the build), 128 threads drop to kProducerRegs and 256 rise to kEpilogueRegs,
+// which sums to exactly the launch's 384 * kLaunchRegs.
+constexpr int kTcThreads = 384;
+constexpr int kLaunchRegs = 168;
+constexpr int kProducerRegs = 56;
+constexpr int kEpilogueRegs = 224;
+static_assert(128 * kProducerRegs + 256 * kEpilogueRegs <= kTcThreads * kLaunchRegs, "register split");
 constexpr int kBM = 128;
 constexpr int kKBlockBytes = 128;
 
@@ -71,6 +80,11 @@ __device__ __forceinline__ void tmem_ld_chunk16(uint32_t taddr, uint32_t (&r)[32
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs)); }
+template <int kRegs>
+__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs)); }
 
 template <int kChunk>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[32]) {
@@ -156,7 +170,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int KB = p.kblocks;
   const int G = p.K / 128;  // scale groups (a8w8)
 
-  if (warp == 0) {
+  if (warp < 4) {
+   setmaxnreg_dec<kProducerRegs>();  // warpgroup 0 hands registers to the epilogue
+   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int it = 0;
@@ -192,7 +208,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int it = 0, acc_it = 0, tile_it = 0;
@@ -254,10 +270,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
       }
     }
+   }
   } else {
-    // ------------------------------------------------------------ epilogue warps 2..9
+    setmaxnreg_inc<kEpilogueRegs>();
+    // ------------------------------------------------------------ epilogue warps 4..11
     const int q = warp & 3;          // TMEM lane quarter this warp may access
-    const int h = (warp - 2) >> 2;   // column half
+    const int h = (warp - 4) >> 2;   // column half
     const int row_in_tile = 32 * q + lane;
     const uint32_t lane_addr = tmem_base + (uint32_t(32 * q) << 16);
     int acc_it = 0, tile_it = 0;
@@ -274,14 +292,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool nb_ok = col0 < p.N;
         const float* asrow = p.a_scale + int64_t(row < p.M ? row : 0) * G;
         const bool row_ok = row < p.M;
+        // a_scale of this row, four groups ahead (L1 hits after the first touch of the row)
         float sa0 = row_ok ? __ldg(asrow + 0) : 0.f;
         float sa1 = (row_ok && KB > 1) ? __ldg(asrow + 1) : 0.f;
+        float sa2 = (row_ok && KB > 2) ? __ldg(asrow + 2) : 0.f;
+        float sa3 = (row_ok && KB > 3) ? __ldg(asrow + 3) : 0.f;
+        float sw0 = nb_ok ? __ldg(p.w_scale + int64_t(nbw) * G) : 0.f;
         for (int kb = 0; kb < KB; ++kb) {
-          const float sa = sa0;
+          const float sc = sa0 * sw0;
           sa0 = sa1;
-          sa1 = (row_ok && kb + 2 < KB) ? __ldg(asrow + kb + 2) : 0.f;
-          const float sw = nb_ok ? __ldg(p.w_scale + int64_t(nbw) * G + kb) : 0.f;
-          const float sc = sa * sw;
+          sa1 = sa2;
+          sa2 = sa3;
+          sa3 = (row_ok && kb + 4 < KB) ? __ldg(asrow + kb + 4) : 0.f;
+          sw0 = (nb_ok && kb + 1 < KB) ? __ldg(p.w_scale + int64_t(nbw) * G + kb + 1) : 0.f;
           const int b = acc_it & 1;
           if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (acc_it >> 1) & 1, abort_flag, &g_status))) {
             ok = false;
@@ -289,17 +312,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           tc_fence_after();
           const uint32_t t_addr = lane_addr + uint32_t(b * BN + h * C::kHalfCols);
+          // TMEM reads double-buffered: chunk c+1 is in flight while chunk c is scaled and
+          // accumulated; the buffer is released as soon as its last chunk has landed
+          uint32_t r0[32], r1[32];
+          tmem_ld<C::kChunk>(t_addr, r0);
+          tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c) {
-            uint32_t r[32];
-            tmem_ld<C::kChunk>(t_addr + c * C::kChunk, r);
-            tmem_ld_wait();
+            uint32_t(&cur)[32] = (c & 1) ? r1 : r0;
+            uint32_t(&nxt)[32] = (c & 1) ? r0 : r1;
+            if (c + 1 < C::kChunks) tmem_ld<C::kChunk>(t_addr + (c + 1) * C::kChunk, nxt);
 #pragma unroll
-            for (int j = 0; j < C::kChunk; ++j) acc[c * C::kChunk + j] = fmaf(__uint_as_float(r[j]), sc, acc[c * C::kChunk + j]);
+            for (int j = 0; j < C::kChunk; ++j)
+              acc[c * C::kChunk + j] = fmaf(__uint_as_float(cur[j]), sc, acc[c * C::kChunk + j]);
+            if (c + 1 < C::kChunks) {
+              tmem_ld_wait();
+              if (c + 2 == C::kChunks) {  // the last chunk is in registers: free the buffer
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty_bar(b));
+              }
+            }
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar(b));
+          if (C::kChunks == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(b));
+          }
           ++acc_it;
         }
         if (!ok) break;
