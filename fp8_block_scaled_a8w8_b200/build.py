@@ -25,7 +25,7 @@ LIB = os.path.join(PKG, "libfp8bs.so")
 INCLUDE = os.path.join(ROOT, "include")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-SOURCES = ["api.cu", "dispatch.cpp", "quant.cu", "gemv.cu", "gemv_tma.cu", "gemm_tc.cu", "tma_host.cu"]
+SOURCES = ["api.cu", "dispatch.cpp", "quant.cu", "gemv.cu", "gemv_tma.cu", "gemv_umma.cu", "gemm_tc.cu", "tma_host.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC]
 

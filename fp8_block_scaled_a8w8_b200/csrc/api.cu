@@ -59,6 +59,7 @@ static size_t op_workspace(int op, int64_t M, int64_t N, int64_t K, const Kernel
   switch (cfg.path) {
     case kPathGemv: return gemv_workspace_bytes(op, M, N, K, cfg);
     case kPathGemvTma: return gemv_tma_workspace_bytes(M, N, K);
+    case kPathGemvUmma: return gemv_umma_workspace_bytes(M, N, K);
     default: return tc_workspace_bytes(op, M, N, K, cfg);
   }
 }
@@ -143,6 +144,9 @@ FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const f
   else if (cfg->path == kPathGemvTma)
     e = launch_gemv_tma_a8w8(A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace,
                              (flags & FP8BS_FLAG_STATIC_WEIGHTS) ? 1 : 0, stream);
+  else if (cfg->path == kPathGemvUmma)
+    e = launch_gemv_umma_a8w8(A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace,
+                              (flags & FP8BS_FLAG_STATIC_WEIGHTS) ? 1 : 0, stream);
   else
     e = launch_tc_a8w8(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream);
   return from_cuda(e);
@@ -198,7 +202,7 @@ FP8BS_API fp8bs_status fp8bs_gemm_bf16(const void* A_bf16, const void* W_bf16, v
 
 FP8BS_API fp8bs_status fp8bs_get_device_status(fp8bs_stream_t stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP8BS_ERR_CUDA;
-  const unsigned int a = take_status_tc(), b = take_status_gemv_tma();
+  const unsigned int a = take_status_tc(), b = take_status_gemv_tma() | take_status_gemv_umma();
   if (a == ~0u || b == ~0u) return FP8BS_ERR_CUDA;
   const unsigned int v = a | b;
   return (v & kStatusTimeout) ? FP8BS_ERR_TIMEOUT : FP8BS_OK;

@@ -29,6 +29,7 @@ static const KernelConfig kConfigs[] = {
     {"a8w8_gemv_d3", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemv, 0, 1, 3},
     {"a8w8_gemv_d4", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemv, 0, 1, 4},
     {"a8w8_gemv_tma", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemvTma, 0, 1, 0},
+    {"a8w8_gemv_umma", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemvUmma, 0, 1, 0},
     {"a8w8_tc_bn128", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 128, 1, 0},
     {"a8w8_tc_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 256, 1, 0},
     {"bf16_gemv_d2", FP8BS_OP_BF16, kPathGemv, 0, 1, 2},
@@ -62,7 +63,7 @@ const KernelConfig* const* list_configs(int op, int* count) {
 const KernelConfig* default_config(int op, int64_t M, int64_t N, int64_t K) {
   (void)K;
   if (op == FP8BS_OP_A8W8_BLOCKSCALE) {
-    if (M <= kGemvMaxM) return find_config(op, "a8w8_gemv_tma");
+    if (M <= kGemvMaxM) return find_config(op, "a8w8_gemv_umma");
     if (N % 256 == 0) return find_config(op, "a8w8_tc_bn256");
     return find_config(op, "a8w8_tc_bn128");
   }
@@ -193,7 +194,8 @@ __attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_set_row(int o
   if (op < 0 || op >= FP8BS_NUM_OPS || M <= 0 || N <= 0 || K <= 0 || !cfg) return FP8BS_ERR_INVALID_ARG;
   const KernelConfig* c = find_config(op, cfg);
   if (!c) return FP8BS_ERR_INVALID_ARG;
-  if ((c->path == kPathGemv || c->path == kPathGemvTma) && M > kGemvMaxM) return FP8BS_ERR_UNSUPPORTED;
+  if ((c->path == kPathGemv || c->path == kPathGemvTma || c->path == kPathGemvUmma) && M > kGemvMaxM)
+    return FP8BS_ERR_UNSUPPORTED;
   State& st = state();
   std::lock_guard<std::mutex> lk(st.mu);
   st.rows[Key{op, M, N, K}] = c;

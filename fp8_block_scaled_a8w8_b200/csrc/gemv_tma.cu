@@ -62,7 +62,10 @@ struct GtCfg {
   static constexpr int kAAlloc = (kABytes + 1023) / 1024 * 1024;  // keeps every tile 1024-byte aligned
   static constexpr int kStageBytes = kWBytes + kAAlloc;
   static constexpr int kStages = (200 * 1024) / kStageBytes > 12 ? 12 : (200 * 1024) / kStageBytes;
-  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 256;
+  // scale staging region: a_scale as [G][8 * NB] (zero past M) then w_scale of the CTA's units
+  static constexpr int kScaleBytes = 24 * 1024;
+  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 + 256 + kScaleBytes;
+  static_assert(kSmemBytes <= 232448, "exceeds the per-CTA shared-memory limit");
 };
 
 struct GtParams {
@@ -96,7 +99,7 @@ __device__ __forceinline__ void gt_store(const GtParams& p, int b, int w, int la
 
 // Finish block b if this CTA was its last contributor (arrival count old == contributors - 1):
 // sum the contributors' partials in CTA order (a fixed order: bit-reproducible results),
-// four loads in flight at a time, store the output, reset the block's counter.
+// kBatch contributors' loads in flight at a time, store the output, reset the block's counter.
 // Contributor cc > cf of block b started its range inside b (its slot 0); the first
 // contributor cf used slot 0 only if its range started exactly at b's first unit, else b
 // was its last block (slot 1).
@@ -112,10 +115,11 @@ __device__ __forceinline__ void gt_finish_block(const GtParams& p, int b, unsign
   for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
     for (int i = 0; i < 4; ++i) sum[nb][i] = 0.f;
-  for (int64_t c0 = cf; c0 <= cl; c0 += 4) {
-    float v[4][NB][4];
+  constexpr int kBatch = NB <= 2 ? 8 : 4;  // 4 * NB * kBatch floats held per thread
+  for (int64_t c0 = cf; c0 <= cl; c0 += kBatch) {
+    float v[kBatch][NB][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < kBatch; ++j) {
       const int64_t cc = c0 + j;
       const int64_t sl = 2 * cc + (cc == cf ? cf_slot : 0);
       const float* src = p.part + (sl * kGtConsumers + w) * (NB * 4 * 32);
@@ -125,7 +129,7 @@ __device__ __forceinline__ void gt_finish_block(const GtParams& p, int b, unsign
         for (int i = 0; i < 4; ++i) v[j][nb][i] = cc <= cl ? __ldcg(src + (nb * 4 + i) * 32 + lane) : 0.f;
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < kBatch; ++j)
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
@@ -135,7 +139,9 @@ __device__ __forceinline__ void gt_finish_block(const GtParams& p, int b, unsign
   if (w == 0 && lane == 0) p.counter[b] = 0u;
 }
 
-template <int NB>
+// kScalesSmem: every CTA's scales fit the staging region (else each unit reads its scales
+// from global memory; only very large K or N get there)
+template <int NB, bool kScalesSmem>
 __global__ void __launch_bounds__(kGtThreads, 1)
     gemv_tma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA, const GtParams p) {
   using C = GtCfg<NB>;
@@ -145,6 +151,7 @@ __global__ void __launch_bounds__(kGtThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(S) * C::kStageBytes);  // full[S], empty[S]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S);
   volatile unsigned* red_slot = reinterpret_cast<volatile unsigned*>(bars + 2 * S) + 1;  // [2]
+  float* sa_s = reinterpret_cast<float*>(smem + size_t(S) * C::kStageBytes + 256);  // [G][8 * NB]
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -248,21 +255,46 @@ __global__ void __launch_bounds__(kGtThreads, 1)
       off_w[c] = uint32_t((16 * w + gid) * 128) + chunk;
       off_a[c] = uint32_t(C::kWBytes + gid * 128) + chunk;
     }
+    // Stage the scales this CTA needs in shared memory: one global round trip here instead
+    // of one per unit on the stream's critical path. a_scale goes in as [G][8 * NB] (zero
+    // for tokens past M, so the loop needs no guard); w_scale is [nblk, G] row-major, so
+    // unit u's weight scale is w_scale[u] and the CTA's are one contiguous run.
+    constexpr int kRows = 8 * NB;
+    float* sw_s = sa_s + G * kRows;
+    if (kScalesSmem) {
+      const int tid = threadIdx.x;  // consumers are threads 0 .. 32 * kGtConsumers - 1
+      for (int i = tid; i < kRows * G; i += 32 * kGtConsumers) {
+        const int t = i / int(G), gg = i - t * int(G);
+        sa_s[gg * kRows + t] = t < p.M ? __ldg(p.a_scale + i) : 0.f;
+      }
+      for (int j = tid; j < u1 - u0; j += 32 * kGtConsumers) sw_s[j] = __ldg(p.w_scale + u0 + j);
+      consumer_bar();
+    }
     int pend0 = -1, pend1 = -1;  // blocks this CTA left partial sums for (at most its first and last)
     int n_pending = 0;
     int it = 0;
     bool aborted = false;
     for (int64_t u = u0; u < u1; ++u, ++it) {
       const int s = it % S;
-      // scales for this unit (L1/L2 hits: a_scale is tiny, w_scale is one word per unit)
-      float sa[NB][2];
+      float sa[NB][2], sw;
+      if (kScalesSmem) {
+        const float* r = sa_s + g * kRows + 2 * tig;
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb) {
-        const int t0 = nb * 8 + 2 * tig;
-        sa[nb][0] = t0 < p.M ? __ldg(p.a_scale + int64_t(t0) * G + g) : 0.f;
-        sa[nb][1] = t0 + 1 < p.M ? __ldg(p.a_scale + int64_t(t0 + 1) * G + g) : 0.f;
+        for (int nb = 0; nb < NB; ++nb) {
+          const float2 v = *reinterpret_cast<const float2*>(r + nb * 8);
+          sa[nb][0] = v.x;
+          sa[nb][1] = v.y;
+        }
+        sw = sw_s[u - u0];
+      } else {
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          const int t0 = nb * 8 + 2 * tig;
+          sa[nb][0] = t0 < p.M ? __ldg(p.a_scale + int64_t(t0) * G + g) : 0.f;
+          sa[nb][1] = t0 + 1 < p.M ? __ldg(p.a_scale + int64_t(t0 + 1) * G + g) : 0.f;
+        }
+        sw = __ldg(p.w_scale + int64_t(b) * G + g);
       }
-      const float sw = __ldg(p.w_scale + int64_t(b) * G + g);
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(full_bar(s), (it / S) & 1, abort_flag, &g_status))) {
         aborted = true;
         break;
@@ -276,30 +308,45 @@ __global__ void __launch_bounds__(kGtThreads, 1)
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) av[nb][c] = *reinterpret_cast<const uint4*>(st + off_a[c] + nb * 8 * 128);
       }
-      float d[NB][4];
+      // A warp works through one unit at a time, so the latency of dependent MMAs is exposed:
+      // the four k slices (c, h) of a token tile accumulate separately (summed below) for
+      // NB <= 2, in two chains for NB = 3; at NB = 4 the register budget leaves one chain per
+      // tile (four independent tiles).
+      constexpr int kChains = NB <= 2 ? 4 : (NB == 3 ? 2 : 1);
+      float d[kChains][NB][4];
 #pragma unroll
-      for (int nb = 0; nb < NB; ++nb)
+      for (int c = 0; c < kChains; ++c)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) d[nb][i] = 0.f;
+        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+          for (int i = 0; i < 4; ++i) d[c][nb][i] = 0.f;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
           const uint32_t a0 = h ? wa[c].z : wa[c].x, a2 = h ? wa[c].w : wa[c].y;
           const uint32_t a1 = h ? wb[c].z : wb[c].x, a3 = h ? wb[c].w : wb[c].y;
 #pragma unroll
           for (int nb = 0; nb < NB; ++nb)
-            mma_e4m3_16832(d[nb], a0, a1, a2, a3, h ? av[nb][c].z : av[nb][c].x, h ? av[nb][c].w : av[nb][c].y);
+            mma_e4m3_16832(d[(2 * h + c) % kChains][nb], a0, a1, a2, a3, h ? av[nb][c].z : av[nb][c].x,
+                           h ? av[nb][c].w : av[nb][c].y);
         }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));  // the MMAs consumed the stage's bytes
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
         const float s0 = sa[nb][0] * sw, s1 = sa[nb][1] * sw;
-        acc[nb][0] = fmaf(d[nb][0], s0, acc[nb][0]);
-        acc[nb][1] = fmaf(d[nb][1], s1, acc[nb][1]);
-        acc[nb][2] = fmaf(d[nb][2], s0, acc[nb][2]);
-        acc[nb][3] = fmaf(d[nb][3], s1, acc[nb][3]);
+        float dd[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          dd[i] = d[0][nb][i];
+          if (kChains >= 2) dd[i] += d[kChains >= 2 ? 1 : 0][nb][i];
+          if (kChains == 4) dd[i] += d[kChains == 4 ? 2 : 0][nb][i] + d[kChains == 4 ? 3 : 0][nb][i];
+        }
+        acc[nb][0] = fmaf(dd[0], s0, acc[nb][0]);
+        acc[nb][1] = fmaf(dd[1], s1, acc[nb][1]);
+        acc[nb][2] = fmaf(dd[2], s0, acc[nb][2]);
+        acc[nb][3] = fmaf(dd[3], s1, acc[nb][3]);
       }
 
       if (g == G - 1 || u == u1 - 1) {
@@ -360,15 +407,15 @@ size_t gemv_tma_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return kCounterBytes + size_t(2) * gt_ctas(M, N, K) * kGtConsumers * nb * 4 * 32 * sizeof(float);
 }
 
-template <int NB>
-static int launch_gt(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out, int64_t M,
+template <int NB, bool kScalesSmem>
+static int launch_gt_impl(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out, int64_t M,
                      int64_t N, int64_t K, void* ws, int static_w, void* stream) {
   using Cc = GtCfg<NB>;
   if ((N + kGtRows - 1) / kGtRows > kMaxCounters) return int(cudaErrorInvalidValue);
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(gemv_tma_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cc::kSmemBytes));
+    attr = cudaFuncSetAttribute(gemv_tma_kernel<NB, kScalesSmem>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cc::kSmemBytes));
   });
   if (attr != cudaSuccess) return int(attr);
   CUtensorMap mw, ma;
@@ -386,7 +433,19 @@ static int launch_gt(const void* A, const float* a_scale, const void* W, const f
   p.static_w = static_w;
   p.counter = static_cast<unsigned*>(ws);
   p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
-  return launch_kernel(gemv_tma_kernel<NB>, dim3(p.n_ctas), dim3(kGtThreads), Cc::kSmemBytes, stream, mw, ma, p);
+  return launch_kernel(gemv_tma_kernel<NB, kScalesSmem>, dim3(p.n_ctas), dim3(kGtThreads), Cc::kSmemBytes, stream, mw, ma, p);
+}
+
+template <int NB>
+static int launch_gt(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out, int64_t M,
+                     int64_t N, int64_t K, void* ws, int static_w, void* stream) {
+  const int64_t G = K / 128;
+  const int64_t units = (N + kGtRows - 1) / kGtRows * G;
+  const int64_t ctas = gt_ctas(M, N, K);
+  const int64_t max_units = (units + ctas - 1) / ctas;
+  if ((G * 8 * NB + max_units) * int64_t(sizeof(float)) <= GtCfg<NB>::kScaleBytes)
+    return launch_gt_impl<NB, true>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
+  return launch_gt_impl<NB, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
 }
 
 int launch_gemv_tma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,

@@ -1,0 +1,442 @@
+// Weight-streaming split-K GEMM for decode M (<= 32) on the 5th-generation tensor cores.
+//
+// Decode reads every weight byte once from HBM and does little arithmetic per byte
+// ([aiter#7752] "[Perf] Retune gfx942 Qwen3.8-27B a8w8 blockscale decode rows for cold
+// weights": in a decode step the weights come from HBM), so all SMs stream their share
+// of W ([mi210 docs/43] section 3: at M = 1 too few workgroups leave the card idle) and
+// the arithmetic must never hold the stream up. The work split is the one of the
+// mma.sync weight-streaming kernel: a unit is one 128-row weight block x one 128-wide K
+// group (exactly one w_scale entry), units are ordered block-major and cut into equal
+// contiguous ranges, one per CTA ("stream-K"), and a block shared by several CTAs is
+// finished by its last contributor, which sums the float32 partials in CTA order (a
+// fixed order: bit-reproducible results).
+//
+// The products run on tcgen05 with the operands swapped ("swap AB"): the weight box is
+// the MMA's A operand (M = 128 weight rows), the token box its B operand (N = 32 token
+// slots; TMA zero-fills the rows past M), both K-major with the 128-byte swizzle the
+// TMA wrote. One thread issues a unit's four K = 32 MMAs into one of eight 32-column
+// TMEM buffers and commits; the epilogue warps take finished buffers with tcgen05.ld
+// (TMEM lane = weight row = thread), multiply the unit's float32 partial by
+// a_scale[token, g] * w_scale[block, g] and accumulate in registers -- the block-scale
+// definition group by group ([cookbook#8]: 128x128 weight blocks, 1x128 activation
+// groups). The tensor core runs up to eight units ahead of the epilogue.
+//
+//   warp 0        TMA producer: per unit one weight box (128 rows x 128 bytes) and one
+//                 token box (32 rows x 128 bytes); with static weights the first ring's
+//                 weight boxes are fetched before the grid-dependency wait
+//   warp 1        TMEM allocator and MMA issuer (one thread)
+//   warps 2..3    only take part in the split-K reduction
+//   warps 4..7    epilogue: warp 4 + q reads TMEM lanes 32q .. 32q + 31
+//
+// The CTA's scales are staged in shared memory once (a_scale as [G][32], zero past M;
+// its run of w_scale, which is [nblk, G] row-major, so unit u's weight scale is
+// w_scale[u]); shapes whose scales do not fit the staging region go to the mma.sync
+// kernel instead.
+//
+// Every wait is bounded (kWaitLimitNs); on expiry the CTA raises its abort flag and the
+// device status word, every role leaves its loop, in-flight TMA copies and MMAs are
+// drained (bounded), TMEM is freed and the CTA exits without publishing partial sums.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fp8bs {
+
+FP8BS_DEFINE_STATUS(gemv_umma)
+
+constexpr int kGuThreads = 256;
+constexpr int kGuRows = 128;                          // weight rows per block = MMA M = TMEM lanes
+constexpr int kGuSlots = 32;                          // token slots = MMA N
+constexpr int kGuBufs = 8;                            // TMEM accumulator buffers
+constexpr int kGuTmemCols = kGuBufs * kGuSlots;       // 256
+constexpr int kGuWBytes = kGuRows * 128;              // 16 KiB weight box
+constexpr int kGuABytes = kGuSlots * 128;             // 4 KiB token box
+constexpr int kGuStageBytes = kGuWBytes + kGuABytes;  // multiple of 1024: every box stays aligned
+constexpr int kGuStages = 10;
+constexpr int kGuBarBytes = 512;
+constexpr int kGuScaleBytes = 24 * 1024;
+constexpr size_t kGuSmemBytes = size_t(kGuStages) * kGuStageBytes + kGuBarBytes + kGuScaleBytes + 1024;
+static_assert(kGuStageBytes % 1024 == 0, "stage alignment");
+static_assert((2 * kGuStages + 2 * kGuBufs + 1) * 8 + 8 * 4 <= kGuBarBytes, "barrier region");
+static_assert(kGuSmemBytes <= 232448, "exceeds the per-CTA shared-memory limit");
+constexpr uint32_t kGuIdesc = make_idesc(kFmtE4M3, kFmtE4M3, kGuRows, kGuSlots);
+
+struct GuParams {
+  const float* a_scale;  // [M, G]
+  const float* w_scale;  // [nblk, G]
+  __nv_bfloat16* out;    // [M, N]
+  int M, N, G, nblk;
+  int n_ctas;
+  int static_w;          // W / w_scale are not written by any kernel still in flight
+  float* part;           // [2 * n_ctas][kGuSlots][kGuRows]
+  unsigned* counter;     // [nblk]
+};
+
+__device__ __forceinline__ int64_t gu_cta_of_unit(int64_t u, int64_t U, int64_t C) { return ((u + 1) * C - 1) / U; }
+
+__device__ __forceinline__ void gu_epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+template <int NT>
+__device__ __forceinline__ void gu_tmem_ld(uint32_t taddr, uint32_t (&r)[NT]) {
+  if constexpr (NT == 8)
+    tmem_ld_32x32b_x8(taddr, r);
+  else if constexpr (NT == 16)
+    tmem_ld_32x32b_x16(taddr, r);
+  else
+    tmem_ld_32x32b_x32(taddr, r);
+}
+
+// Finish block b if this CTA was its last contributor (arrival count old == contributors
+// - 1): all 256 threads sum the contributors' partials in CTA order, kB contributors'
+// loads in flight at a time, store the bf16 output and reset the block's counter.
+// Thread tid owns weight row tid % 128 and tokens tid / 128 + 2j. Contributor cc > cf
+// started its range inside b (its slot 0); the first contributor cf used slot 0 only if
+// its range started exactly at b's first unit, else b was its last block (slot 1).
+template <int NT>
+__device__ __forceinline__ void gu_finish_block(const GuParams& p, int b, unsigned old, int64_t U, int64_t Cn,
+                                                int64_t G) {
+  const int64_t cf = gu_cta_of_unit(int64_t(b) * G, U, Cn);
+  const int64_t cl = gu_cta_of_unit(int64_t(b + 1) * G - 1, U, Cn);
+  if (old != unsigned(cl - cf)) return;
+  const int cf_slot = (U * cf / Cn >= int64_t(b) * G) ? 0 : 1;
+  constexpr int kE = NT * kGuRows / kGuThreads;  // elements per thread
+  constexpr int kB = kE >= 16 ? 4 : 8;
+  const int tid = threadIdx.x;
+  const int r = tid & (kGuRows - 1);
+  const int t0 = tid >> 7;
+  float sum[kE];
+#pragma unroll
+  for (int j = 0; j < kE; ++j) sum[j] = 0.f;
+  for (int64_t c0 = cf; c0 <= cl; c0 += kB) {
+    float v[kB][kE];
+#pragma unroll
+    for (int jj = 0; jj < kB; ++jj) {
+      const int64_t cc = c0 + jj;
+      const int64_t sl = 2 * cc + (cc == cf ? cf_slot : 0);
+      const float* src = p.part + sl * (kGuSlots * kGuRows) + r;
+#pragma unroll
+      for (int j = 0; j < kE; ++j) {
+        const int t = t0 + 2 * j;
+        v[jj][j] = (cc <= cl && t < p.M) ? __ldcg(src + t * kGuRows) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int jj = 0; jj < kB; ++jj)
+#pragma unroll
+      for (int j = 0; j < kE; ++j) sum[j] += v[jj][j];
+  }
+  const int n = b * kGuRows + r;
+  if (n < p.N) {
+#pragma unroll
+    for (int j = 0; j < kE; ++j) {
+      const int t = t0 + 2 * j;
+      if (t < p.M) p.out[int64_t(t) * p.N + n] = __float2bfloat16_rn(sum[j]);
+    }
+  }
+  if (tid == 0) p.counter[b] = 0u;
+}
+
+// NT: token columns the epilogue reads per unit (8, 16 or 32 >= M).
+template <int NT>
+__global__ void __launch_bounds__(kGuThreads, 1)
+    gemv_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA, const GuParams p) {
+  constexpr int S = kGuStages;
+  constexpr int B = kGuBufs;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(S) * kGuStageBytes);  // full[S] empty[S] tfull[B] tempty[B] drain
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * B + 1);
+  uint32_t* tmem_slot = misc;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile int* pend_s = reinterpret_cast<volatile int*>(misc + 2);             // n_pending, block 0, block 1
+  volatile unsigned* red_slot = reinterpret_cast<volatile unsigned*>(misc + 5);  // [2]
+  float* sa_s = reinterpret_cast<float*>(smem + size_t(S) * kGuStageBytes + kGuBarBytes);  // [G][kGuSlots]
+
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t G = p.G;
+  const int64_t U = int64_t(p.nblk) * G;
+  const int64_t Cn = p.n_ctas;
+  const int cta = blockIdx.x;
+  const int64_t u0 = U * cta / Cn, u1 = U * (cta + 1) / Cn;
+  const int n_units = int(u1 - u0);
+  const int first_blk = int(u0 / G);
+  float* sw_s = sa_s + G * kGuSlots;  // [n_units]
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + S + s); };
+  auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * S + b); };
+  auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * S + B + b); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * S + 2 * B);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < B; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    pend_s[0] = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmA);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kGuTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int last_it[kGuStages];
+      for (int s = 0; s < S; ++s) last_it[s] = -1;
+      int b = first_blk, g = int(u0 - int64_t(first_blk) * G);
+      int it = 0;
+      if (p.static_w) {
+        // The weights are not produced by an earlier kernel: fetch the first ring's worth
+        // of weight boxes before waiting for the previous kernel, overlapping its tail.
+        const int pre = n_units < S ? n_units : S;
+        int pb = b, pg = g;
+        for (int j = 0; j < pre; ++j) {
+          const uint32_t dst = smem_u32(smem + size_t(j) * kGuStageBytes);
+          mbar_arrive_expect_tx(full_bar(j), kGuStageBytes);
+          tma_load_2d(dst, &tmW, full_bar(j), pg * 128, pb * kGuRows);
+          if (++pg == G) {
+            pg = 0;
+            ++pb;
+          }
+        }
+        pdl_wait();
+        for (int j = 0; j < pre; ++j, ++it) {
+          const uint32_t dst = smem_u32(smem + size_t(j) * kGuStageBytes);
+          tma_load_2d(dst + kGuWBytes, &tmA, full_bar(j), g * 128, 0);
+          last_it[j] = it;
+          if (++g == G) {
+            g = 0;
+            ++b;
+          }
+        }
+      } else {
+        pdl_wait();
+      }
+      for (; it < n_units; ++it) {
+        const int s = it % S;
+        if (!mbar_wait_bounded(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, &g_status)) break;
+        const uint32_t dst = smem_u32(smem + size_t(s) * kGuStageBytes);
+        mbar_arrive_expect_tx(full_bar(s), kGuStageBytes);
+        tma_load_2d(dst, &tmW, full_bar(s), g * 128, b * kGuRows);
+        tma_load_2d(dst + kGuWBytes, &tmA, full_bar(s), g * 128, 0);
+        last_it[s] = it;
+        if (++g == G) {
+          g = 0;
+          ++b;
+        }
+      }
+      for (int s = 0; s < S; ++s) {  // drain (bounded): every issued copy has landed
+        if (last_it[s] < 0) continue;
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(full_bar(s), (last_it[s] / S) & 1))
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, kStatusTimeout);
+            break;
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool issued = false;
+      for (int it = 0; it < n_units; ++it) {
+        const int s = it % S;
+        if (!mbar_wait_bounded(full_bar(s), (it / S) & 1, abort_flag, &g_status)) break;
+        const int buf = it % B;
+        if (!mbar_wait_bounded(tempty_bar(buf), ((it / B) & 1) ^ 1, abort_flag, &g_status)) break;
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + size_t(s) * kGuStageBytes);
+        const uint64_t adesc = sw128_kmajor_desc(st);
+        const uint64_t bdesc = sw128_kmajor_desc(st + kGuWBytes);
+        const uint32_t d_tmem = tmem_base + uint32_t(buf * kGuSlots);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) umma_f8f6f4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kGuIdesc, kk > 0);
+        issued = true;
+        umma_commit(empty_bar(s));    // the stage's bytes are consumed once these MMAs complete
+        umma_commit(tfull_bar(buf));  // the unit's partial is in TMEM
+      }
+      if (issued) {  // drain: every MMA issued by this thread has completed once drain_bar flips
+        umma_commit(drain_bar);
+        const unsigned long long t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain_bar, 0))
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, kStatusTimeout);
+            break;
+          }
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue warps 4..7
+    pdl_wait();  // activations' scales and the workspace come from earlier kernels
+    const int q = warp - 4;
+    const int r = 32 * q + lane;  // weight row within the block = TMEM lane
+    const uint32_t lane_addr = tmem_base + (uint32_t(32 * q) << 16);
+    const int et = threadIdx.x - 128;
+    for (int i = et; i < kGuSlots * int(G); i += 128) {
+      const int t = i / int(G), gg = i - t * int(G);
+      sa_s[gg * kGuSlots + t] = t < p.M ? __ldg(p.a_scale + i) : 0.f;
+    }
+    for (int j = et; j < n_units; j += 128) sw_s[j] = __ldg(p.w_scale + u0 + j);
+    gu_epilogue_bar();
+
+    float acc[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+    int b = first_blk, g = int(u0 - int64_t(first_blk) * G);
+    int n_pending = 0, pend0 = -1, pend1 = -1;
+    for (int it = 0; it < n_units; ++it) {
+      const int buf = it % B;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(buf), (it / B) & 1, abort_flag, &g_status))) break;
+      tc_fence_after();
+      uint32_t d[NT];
+      gu_tmem_ld<NT>(lane_addr + uint32_t(buf * kGuSlots), d);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(buf));  // the buffer may take the next unit
+      const float sw = sw_s[it];
+      const float* sa = sa_s + g * kGuSlots;
+#pragma unroll
+      for (int t = 0; t < NT; t += 4) {
+        const float4 s4 = *reinterpret_cast<const float4*>(sa + t);
+        acc[t + 0] = fmaf(__uint_as_float(d[t + 0]), s4.x * sw, acc[t + 0]);
+        acc[t + 1] = fmaf(__uint_as_float(d[t + 1]), s4.y * sw, acc[t + 1]);
+        acc[t + 2] = fmaf(__uint_as_float(d[t + 2]), s4.z * sw, acc[t + 2]);
+        acc[t + 3] = fmaf(__uint_as_float(d[t + 3]), s4.w * sw, acc[t + 3]);
+      }
+      if (g == G - 1 || it == n_units - 1) {
+        // ---- block b ends here (or the CTA's range does)
+        const bool whole = int64_t(b) * G >= u0 && g == G - 1;
+        if (whole) {
+          const int n = b * kGuRows + r;
+          if (n < p.N) {
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+              if (t < p.M) p.out[int64_t(t) * p.N + n] = __float2bfloat16_rn(acc[t]);
+          }
+        } else {
+          // partial sum: a plain store now, published after the loop
+          const int slot = 2 * cta + (b == first_blk ? 0 : 1);
+          float* dst = p.part + int64_t(slot) * (kGuSlots * kGuRows) + r;
+#pragma unroll
+          for (int t = 0; t < NT; ++t)
+            if (t < p.M) __stcg(dst + t * kGuRows, acc[t]);
+          if (n_pending == 0)
+            pend0 = b;
+          else
+            pend1 = b;
+          ++n_pending;
+        }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+      }
+      if (++g == G) {
+        g = 0;
+        ++b;
+      }
+    }
+    if (threadIdx.x == 128) {
+      pend_s[1] = pend0;
+      pend_s[2] = pend1;
+      pend_s[0] = n_pending;
+    }
+  }
+
+  // ---- every warp: free TMEM, publish the partial sums, finish the blocks this CTA completes
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();  // TMEM reads, partial stores and the pending list are complete
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kGuTmemCols);
+  }
+  pdl_wait();  // warps 1..3 have not waited yet; they write the workspace and the output below
+  const int n_pending = pend_s[0];
+  const bool aborted = *abort_flag != 0;
+  if (threadIdx.x < n_pending)
+    red_slot[threadIdx.x] = aborted ? 0u : atom_add_acq_rel_gpu(p.counter + pend_s[1 + threadIdx.x], 1u);
+  __syncthreads();
+  if (!aborted) {
+    if (n_pending > 0) gu_finish_block<NT>(p, pend_s[1], red_slot[0], U, Cn, G);
+    if (n_pending > 1) gu_finish_block<NT>(p, pend_s[2], red_slot[1], U, Cn, G);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+static int gu_ctas(int64_t N, int64_t K) {
+  const int64_t units = ((N + kGuRows - 1) / kGuRows) * (K / 128);
+  return int(std::min<int64_t>(device_sm_count(), units));
+}
+
+static bool gu_scales_fit(int64_t N, int64_t K) {
+  const int64_t G = K / 128;
+  const int64_t units = ((N + kGuRows - 1) / kGuRows) * G;
+  const int64_t ctas = gu_ctas(N, K);
+  const int64_t max_units = (units + ctas - 1) / ctas;
+  return (G * kGuSlots + max_units) * int64_t(sizeof(float)) <= kGuScaleBytes;
+}
+
+size_t gemv_umma_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  const size_t own = kCounterBytes + size_t(2) * gu_ctas(N, K) * kGuSlots * kGuRows * sizeof(float);
+  return std::max(own, gemv_tma_workspace_bytes(M, N, K));  // shapes whose scales do not fit take that kernel
+}
+
+template <int NT>
+static int launch_gu(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out, int64_t M,
+                     int64_t N, int64_t K, void* ws, int static_w, void* stream) {
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(gemv_umma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGuSmemBytes));
+  });
+  if (attr != cudaSuccess) return int(attr);
+  CUtensorMap mw, ma;
+  if (!make_tma_2d_kmajor(&mw, W, true, N, K, kGuRows) || !make_tma_2d_kmajor(&ma, A, true, M, K, kGuSlots))
+    return int(cudaErrorInvalidValue);
+  GuParams p{};
+  p.a_scale = a_scale;
+  p.w_scale = w_scale;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.M = int(M);
+  p.N = int(N);
+  p.G = int(K / 128);
+  p.nblk = int((N + kGuRows - 1) / kGuRows);
+  p.n_ctas = gu_ctas(N, K);
+  p.static_w = static_w;
+  p.counter = static_cast<unsigned*>(ws);
+  p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
+  return launch_kernel(gemv_umma_kernel<NT>, dim3(p.n_ctas), dim3(kGuThreads), kGuSmemBytes, stream, mw, ma, p);
+}
+
+int launch_gemv_umma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
+                          int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream) {
+  if (M < 1 || M > kGemvMaxM || (N + kGuRows - 1) / kGuRows > kMaxCounters) return int(cudaErrorInvalidValue);
+  if (!gu_scales_fit(N, K))
+    return launch_gemv_tma_a8w8(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
+  if (M <= 8) return launch_gu<8>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
+  if (M <= 16) return launch_gu<16>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
+  return launch_gu<32>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
+}
+
+}  // namespace fp8bs

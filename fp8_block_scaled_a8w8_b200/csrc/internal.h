@@ -18,6 +18,7 @@ enum Path : int {
   kPathGemv = 0,  // weight-streaming split-K kernel (mma.sync, small M)
   kPathTc = 1,    // tcgen05/TMEM tensor-core kernel fed by TMA
   kPathGemvTma = 2,  // weight-streaming split-K kernel fed by TMA (mma.sync, small M)
+  kPathGemvUmma = 3,  // weight-streaming split-K kernel fed by TMA, tcgen05 products (small M)
 };
 
 // One kernel configuration a dispatch-table row can name.
@@ -52,6 +53,7 @@ constexpr int64_t kGemvMaxM = 32;
 // wait (~0u on a CUDA error).
 unsigned int take_status_tc();
 unsigned int take_status_gemv_tma();
+unsigned int take_status_gemv_umma();
 
 // Device properties, cached per device.
 int device_sm_count();
@@ -69,6 +71,10 @@ int launch_gemv_bf16(const KernelConfig& cfg, const void* A, const void* W, void
 size_t gemv_tma_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int launch_gemv_tma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
                          int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream);
+
+size_t gemv_umma_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int launch_gemv_umma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
+                          int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream);
 
 // Launch a kernel on a stream with programmatic stream serialisation (PDL) unless the
 // environment sets FP8BS_PDL=0. Returns the cudaError_t of the launch as int.

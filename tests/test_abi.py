@@ -79,7 +79,7 @@ def test_c_dispatch_walk_matches_page_examples(golden_dir):
             pm, cfg = fb.dispatch_lookup(fb.OP_A8W8_BLOCKSCALE, int(m), 5120, 6144)
             assert pm == (None if want == "miss" else int(want)), (table, m, want, pm)
             if pm is None:  # a miss runs the shape's default configuration
-                assert cfg == ("a8w8_gemv_tma" if int(m) <= 32 else "a8w8_tc_bn256")
+                assert cfg == ("a8w8_gemv_umma" if int(m) <= 32 else "a8w8_tc_bn256")
     finally:
         fb.dispatch_reset_table(keep_builtin=True)
 

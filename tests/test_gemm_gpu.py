@@ -51,17 +51,28 @@ def test_gemv_path_parity(M, N, K):
     check_a8w8(_run(*case), *case)
 
 
-@pytest.mark.parametrize("cfg", ["a8w8_gemv_d2", "a8w8_gemv_d3", "a8w8_gemv_d4", "a8w8_gemv_tma"])
+@pytest.mark.parametrize("cfg", ["a8w8_gemv_d2", "a8w8_gemv_d3", "a8w8_gemv_d4", "a8w8_gemv_tma", "a8w8_gemv_umma"])
 @pytest.mark.parametrize("M", [1, 7, 16, 25])
 def test_gemv_depths(cfg, M):
     case = _raw_case(M, 400, 1408, seed=M + 77)
     check_a8w8(_run(*case, cfg=cfg), *case)
 
 
-@pytest.mark.parametrize("cfg", ["a8w8_gemv_d4", "a8w8_gemv_tma"])
+@pytest.mark.parametrize("cfg", ["a8w8_gemv_d4", "a8w8_gemv_tma", "a8w8_gemv_umma"])
 @pytest.mark.parametrize("M,N,K", [(1, 16, 128), (5, 144, 128), (32, 34816, 5120), (12, 5120, 6144), (2, 130 * 16, 3968)])
 def test_gemv_kernels_shapes(cfg, M, N, K):
     case = _raw_case(M, N, K, seed=M + N + K)
+    check_a8w8(_run(*case, cfg=cfg), *case)
+
+
+# The weight-streaming kernels stage each CTA's scales in a 24 KiB shared-memory region;
+# K this large (a_scale of the token slots x K / 128 groups no longer fits) takes the
+# mma.sync kernel's per-unit global-load variant (the tcgen05 kernel hands such shapes
+# to it).
+@pytest.mark.parametrize("cfg", ["a8w8_gemv_tma", "a8w8_gemv_umma"])
+@pytest.mark.parametrize("M,N,K", [(1, 32, 98432), (8, 16, 98432), (32, 48, 24704), (17, 16, 32896)])
+def test_gemv_scales_not_staged(cfg, M, N, K):
+    case = _raw_case(M, N, K, seed=M + N + K + 5)
     check_a8w8(_run(*case, cfg=cfg), *case)
 
 
@@ -185,7 +196,7 @@ def test_workspace_shared_across_shapes():
         torch.cuda.synchronize()
         check_a8w8(y, *case)
     # the same sequence again on the now-used workspace: bit-identical outputs
-    for cfg in ("a8w8_gemv_d4", "a8w8_gemv_tma"):
+    for cfg in ("a8w8_gemv_d4", "a8w8_gemv_tma", "a8w8_gemv_umma"):
         fb.dispatch_set_row(OP, 9, 2048, 1024, cfg)
         try:
             case = _raw_case(9, 2048, 1024, seed=102)
