@@ -14,24 +14,25 @@
 // The products run on tcgen05 with the operands swapped ("swap AB"): the weight box is
 // the MMA's A operand (M = 128 weight rows), the token box its B operand (N = 32 token
 // slots; TMA zero-fills the rows past M), both K-major with the 128-byte swizzle the
-// TMA wrote. One thread issues a unit's four K = 32 MMAs into one of eight 32-column
-// TMEM buffers and commits; the epilogue warps take finished buffers with tcgen05.ld
+// TMA wrote. An issuing thread issues a unit's four K = 32 MMAs into one of eight
+// 32-column TMEM buffers and commits; the epilogue warps take finished buffers with tcgen05.ld
 // (TMEM lane = weight row = thread), multiply the unit's float32 partial by
 // a_scale[token, g] * w_scale[block, g] and accumulate in registers -- the block-scale
 // definition group by group ([cookbook#8]: 128x128 weight blocks, 1x128 activation
 // groups). The tensor core runs up to eight units ahead of the epilogue.
 //
 //   warp 0        TMA producer: per unit one weight box (128 rows x 128 bytes) and one
-//                 token box (32 rows x 128 bytes); with static weights the first ring's
+//                 token box (32 rows x 128 bytes); with static weights the first few
 //                 weight boxes are fetched before the grid-dependency wait
-//   warp 1        TMEM allocator and MMA issuer (one thread)
-//   warps 2..3    only take part in the split-K reduction
+//   warp 1        TMEM allocator; lane 0 issues the MMAs of even units
+//   warp 2        lane 0 issues the MMAs of odd units
+//   warp 3        only takes part in the split-K reduction
 //   warps 4..7    epilogue: warp 4 + q reads TMEM lanes 32q .. 32q + 31
 //
-// The CTA's scales are staged in shared memory once (a_scale as [G][32], zero past M;
-// its run of w_scale, which is [nblk, G] row-major, so unit u's weight scale is
-// w_scale[u]); shapes whose scales do not fit the staging region go to the mma.sync
-// kernel instead.
+// The CTA's scales are staged in shared memory once (a_scale as [G][NT], NT >= M token
+// columns, zero past M; its run of w_scale, which is [nblk, G] row-major, so unit u's
+// weight scale is w_scale[u]); shapes whose scales do not fit the staging region go to
+// the mma.sync kernel instead.
 //
 // Every wait is bounded (kWaitLimitNs); on expiry the CTA raises its abort flag and the
 // device status word, every role leaves its loop, in-flight TMA copies and MMAs are
@@ -56,15 +57,32 @@ constexpr int kGuSlots = 32;                          // token slots = MMA N
 constexpr int kGuBufs = 8;                            // TMEM accumulator buffers
 constexpr int kGuTmemCols = kGuBufs * kGuSlots;       // 256
 constexpr int kGuWBytes = kGuRows * 128;              // 16 KiB weight box
-constexpr int kGuABytes = kGuSlots * 128;             // 4 KiB token box
+constexpr int kGuABytes = kGuSlots * 128;             // 4 KiB token slots per stage
 constexpr int kGuStageBytes = kGuWBytes + kGuABytes;  // multiple of 1024: every box stays aligned
-constexpr int kGuStages = 10;
+// Two CTAs fit on an SM (shared memory, registers, 2 x 256 TMEM columns), so the next
+// call's CTAs become resident while this call's are still streaming and fetch their first
+// weight boxes during its tail: the HBM stream does not pause between calls.
+constexpr int kGuCtasPerSm = 2;
+constexpr int kGuStages = 5;
+// Weight boxes fetched before the grid-dependency wait (static weights). Each SM's
+// requests are served roughly in issue order, so everything issued after the wait (the
+// token boxes, the activation scales) lands only once these have: fetch about what
+// the gap before the wait can absorb, not the whole ring.
+constexpr int kGuPrefetch = 4;
+// MMA issuing threads (lane 0 of warps 1 .. kGuIssuers): issuer i takes the units with
+// it % kGuIssuers == i. One thread spends longer issuing a unit's MMAs, waits and commits
+// than the HBM needs to deliver the unit's 16 KiB; two keep up.
+constexpr int kGuIssuers = 2;
 constexpr int kGuBarBytes = 512;
-constexpr int kGuScaleBytes = 24 * 1024;
+constexpr int kGuScaleBytes = 8 * 1024;
 constexpr size_t kGuSmemBytes = size_t(kGuStages) * kGuStageBytes + kGuBarBytes + kGuScaleBytes + 1024;
 static_assert(kGuStageBytes % 1024 == 0, "stage alignment");
-static_assert((2 * kGuStages + 2 * kGuBufs + 1) * 8 + 8 * 4 <= kGuBarBytes, "barrier region");
-static_assert(kGuSmemBytes <= 232448, "exceeds the per-CTA shared-memory limit");
+static_assert((2 * kGuStages + 2 * kGuBufs + kGuIssuers) * 8 + 8 * 4 <= kGuBarBytes, "barrier region (misc: 8 words)");
+static_assert(kGuBufs % kGuIssuers == 0, "a TMEM buffer always belongs to the same issuer");
+static_assert(kGuIssuers >= 1 && kGuIssuers <= 2, "issuers are lane 0 of warps 1 and 2");
+static_assert(kGuCtasPerSm * (kGuSmemBytes + 1024) <= 233472, "two CTAs must fit an SM's shared memory");
+static_assert(kGuCtasPerSm * kGuTmemCols <= 512, "two CTAs must fit an SM's TMEM");
+static_assert(kGuPrefetch <= kGuStages, "prefetch within the ring");
 constexpr uint32_t kGuIdesc = make_idesc(kFmtE4M3, kFmtE4M3, kGuRows, kGuSlots);
 
 struct GuParams {
@@ -81,6 +99,10 @@ struct GuParams {
 __device__ __forceinline__ int64_t gu_cta_of_unit(int64_t u, int64_t U, int64_t C) { return ((u + 1) * C - 1) / U; }
 
 __device__ __forceinline__ void gu_epilogue_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Ordering barrier between the epilogue's weight-scale loads and the producer's prefetch
+// (128 epilogue threads arrive, the producer warp's 32 wait).
+__device__ __forceinline__ void gu_order_bar_arrive() { asm volatile("bar.arrive 2, 160;" ::: "memory"); }
+__device__ __forceinline__ void gu_order_bar_sync() { asm volatile("bar.sync 2, 160;" ::: "memory"); }
 
 template <int NT>
 __device__ __forceinline__ void gu_tmem_ld(uint32_t taddr, uint32_t (&r)[NT]) {
@@ -144,19 +166,23 @@ __device__ __forceinline__ void gu_finish_block(const GuParams& p, int b, unsign
 
 // NT: token columns the epilogue reads per unit (8, 16 or 32 >= M).
 template <int NT>
-__global__ void __launch_bounds__(kGuThreads, 1)
+__global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
     gemv_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA, const GuParams p) {
   constexpr int S = kGuStages;
   constexpr int B = kGuBufs;
+  // The token box has NT rows (rows past M read as zero); MMA column n depends only on
+  // token row n, so slots NT..31 may hold anything: their columns are never read.
+  constexpr uint32_t kTx = kGuWBytes + NT * 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(S) * kGuStageBytes);  // full[S] empty[S] tfull[B] tempty[B] drain
-  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * B + 1);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * B + kGuIssuers);
   uint32_t* tmem_slot = misc;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* pend_s = reinterpret_cast<volatile int*>(misc + 2);             // n_pending, block 0, block 1
   volatile unsigned* red_slot = reinterpret_cast<volatile unsigned*>(misc + 5);  // [2]
-  float* sa_s = reinterpret_cast<float*>(smem + size_t(S) * kGuStageBytes + kGuBarBytes);  // [G][kGuSlots]
+  volatile int* passed = reinterpret_cast<volatile int*>(misc + 7);  // units whose full-barrier wait has passed
+  float* sa_s = reinterpret_cast<float*>(smem + size_t(S) * kGuStageBytes + kGuBarBytes);  // [G][NT]
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -167,12 +193,27 @@ __global__ void __launch_bounds__(kGuThreads, 1)
   const int64_t u0 = U * cta / Cn, u1 = U * (cta + 1) / Cn;
   const int n_units = int(u1 - u0);
   const int first_blk = int(u0 / G);
-  float* sw_s = sa_s + G * kGuSlots;  // [n_units]
+  float* sw_s = sa_s + G * NT;  // [n_units]
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
   auto empty_bar = [&](int s) { return smem_u32(bars + S + s); };
   auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * S + b); };
   auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * S + B + b); };
-  const uint32_t drain_bar = smem_u32(bars + 2 * S + 2 * B);
+  auto drain_bar = [&](int i) { return smem_u32(bars + 2 * S + 2 * B + i); };
+  // Bounded spin until units 0 .. it-1 have passed their full-barrier wait.
+  auto wait_passed = [&](int it) {
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t i = 1; *passed < it; ++i) {
+      if ((i & 63u) == 0) {
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          atomicOr(&g_status, kStatusTimeout);
+          return false;
+        }
+      }
+    }
+    return true;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -183,9 +224,10 @@ __global__ void __launch_bounds__(kGuThreads, 1)
       mbar_init(tfull_bar(b), 1);
       mbar_init(tempty_bar(b), 4);  // one arrival per epilogue warp
     }
-    mbar_init(drain_bar, 1);
+    for (int i = 0; i < kGuIssuers; ++i) mbar_init(drain_bar(i), 1);
     *abort_flag = 0;
     pend_s[0] = 0;
+    *passed = 0;
     fence_barrier_init();
     prefetch_tensormap(&tmW);
     prefetch_tensormap(&tmA);
@@ -201,6 +243,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    if (p.static_w) gu_order_bar_sync();  // the epilogue's w_scale requests go out first
     if (lane == 0) {
       int last_it[kGuStages];
       for (int s = 0; s < S; ++s) last_it[s] = -1;
@@ -209,11 +252,11 @@ __global__ void __launch_bounds__(kGuThreads, 1)
       if (p.static_w) {
         // The weights are not produced by an earlier kernel: fetch the first ring's worth
         // of weight boxes before waiting for the previous kernel, overlapping its tail.
-        const int pre = n_units < S ? n_units : S;
+        const int pre = n_units < kGuPrefetch ? n_units : kGuPrefetch;
         int pb = b, pg = g;
         for (int j = 0; j < pre; ++j) {
           const uint32_t dst = smem_u32(smem + size_t(j) * kGuStageBytes);
-          mbar_arrive_expect_tx(full_bar(j), kGuStageBytes);
+          mbar_arrive_expect_tx(full_bar(j), kTx);
           tma_load_2d(dst, &tmW, full_bar(j), pg * 128, pb * kGuRows);
           if (++pg == G) {
             pg = 0;
@@ -237,7 +280,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         const int s = it % S;
         if (!mbar_wait_bounded(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, &g_status)) break;
         const uint32_t dst = smem_u32(smem + size_t(s) * kGuStageBytes);
-        mbar_arrive_expect_tx(full_bar(s), kGuStageBytes);
+        mbar_arrive_expect_tx(full_bar(s), kTx);
         tma_load_2d(dst, &tmW, full_bar(s), g * 128, b * kGuRows);
         tma_load_2d(dst + kGuWBytes, &tmA, full_bar(s), g * 128, 0);
         last_it[s] = it;
@@ -256,13 +299,20 @@ __global__ void __launch_bounds__(kGuThreads, 1)
           }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= 1 && warp <= kGuIssuers) {
+    // ------------------------------------------------------------ MMA issuers
     if (lane == 0) {
+      const int me = warp - 1;
       bool issued = false;
-      for (int it = 0; it < n_units; ++it) {
+      for (int it = me; it < n_units; it += kGuIssuers) {
         const int s = it % S;
+        // Units pass their full-barrier wait in unit order: an issuer that ran a whole ring
+        // ahead of the other would otherwise test stage s's barrier while it still holds an
+        // older phase of the same parity and take stale bytes. (Stages and TMEM buffers are
+        // then also reused strictly in order.)
+        if (kGuIssuers > 1 && !wait_passed(it)) break;
         if (!mbar_wait_bounded(full_bar(s), (it / S) & 1, abort_flag, &g_status)) break;
+        if (kGuIssuers > 1) *passed = it + 1;
         const int buf = it % B;
         if (!mbar_wait_bounded(tempty_bar(buf), ((it / B) & 1) ^ 1, abort_flag, &g_status)) break;
         tc_fence_after();
@@ -277,9 +327,9 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         umma_commit(tfull_bar(buf));  // the unit's partial is in TMEM
       }
       if (issued) {  // drain: every MMA issued by this thread has completed once drain_bar flips
-        umma_commit(drain_bar);
+        umma_commit(drain_bar(me));
         const unsigned long long t0 = globaltimer_ns();
-        while (!mbar_try_wait(drain_bar, 0))
+        while (!mbar_try_wait(drain_bar(me), 0))
           if (globaltimer_ns() - t0 > kWaitLimitNs) {
             atomicOr(&g_status, kStatusTimeout);
             break;
@@ -288,16 +338,44 @@ __global__ void __launch_bounds__(kGuThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue warps 4..7
-    pdl_wait();  // activations' scales and the workspace come from earlier kernels
     const int q = warp - 4;
     const int r = 32 * q + lane;  // weight row within the block = TMEM lane
     const uint32_t lane_addr = tmem_base + (uint32_t(32 * q) << 16);
     const int et = threadIdx.x - 128;
-    for (int i = et; i < kGuSlots * int(G); i += 128) {
-      const int t = i / int(G), gg = i - t * int(G);
-      sa_s[gg * kGuSlots + t] = t < p.M ? __ldg(p.a_scale + i) : 0.f;
+    // Stage the scales: the CTA's run of w_scale (static weights: requested before the
+    // producer's weight prefetch, which waits on the ordering barrier) and a_scale as
+    // [G][NT] (written by the previous kernel: after the grid-dependency wait), each
+    // thread's loads issued together.
+    if (p.static_w) {
+      float v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) v[k] = et + 128 * k < n_units ? __ldg(p.w_scale + u0 + et + 128 * k) : 0.f;
+      gu_order_bar_arrive();
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (et + 128 * k < n_units) sw_s[et + 128 * k] = v[k];
+      for (int j = et + 512; j < n_units; j += 128) sw_s[j] = __ldg(p.w_scale + u0 + j);
+      pdl_wait();  // activation scales and the workspace come from earlier kernels
+    } else {
+      pdl_wait();  // so may the weight scales
+      for (int j = et; j < n_units; j += 128) sw_s[j] = __ldg(p.w_scale + u0 + j);
     }
-    for (int j = et; j < n_units; j += 128) sw_s[j] = __ldg(p.w_scale + u0 + j);
+    constexpr int kPer = 8;
+    for (int base = 0; base < NT * int(G); base += 128 * kPer) {
+      float v[kPer];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int i = base + 128 * k + et;  // = t * G + gg
+        const int t = i / int(G);
+        v[k] = (i < NT * int(G) && t < p.M) ? __ldg(p.a_scale + i) : 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int i = base + 128 * k + et;
+        const int t = i / int(G), gg = i - t * int(G);
+        if (i < NT * int(G)) sa_s[gg * NT + t] = v[k];
+      }
+    }
     gu_epilogue_bar();
 
     float acc[NT];
@@ -316,7 +394,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(buf));  // the buffer may take the next unit
       const float sw = sw_s[it];
-      const float* sa = sa_s + g * kGuSlots;
+      const float* sa = sa_s + g * NT;
 #pragma unroll
       for (int t = 0; t < NT; t += 4) {
         const float4 s4 = *reinterpret_cast<const float4*>(sa + t);
@@ -389,12 +467,13 @@ static int gu_ctas(int64_t N, int64_t K) {
   return int(std::min<int64_t>(device_sm_count(), units));
 }
 
-static bool gu_scales_fit(int64_t N, int64_t K) {
+static bool gu_scales_fit(int64_t M, int64_t N, int64_t K) {
   const int64_t G = K / 128;
   const int64_t units = ((N + kGuRows - 1) / kGuRows) * G;
   const int64_t ctas = gu_ctas(N, K);
   const int64_t max_units = (units + ctas - 1) / ctas;
-  return (G * kGuSlots + max_units) * int64_t(sizeof(float)) <= kGuScaleBytes;
+  const int64_t nt = M <= 8 ? 8 : M <= 16 ? 16 : 32;
+  return (G * nt + max_units) * int64_t(sizeof(float)) <= kGuScaleBytes;
 }
 
 size_t gemv_umma_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -409,10 +488,13 @@ static int launch_gu(const void* A, const float* a_scale, const void* W, const f
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
     attr = cudaFuncSetAttribute(gemv_umma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGuSmemBytes));
+    if (attr == cudaSuccess)
+      attr = cudaFuncSetAttribute(gemv_umma_kernel<NT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  int(cudaSharedmemCarveoutMaxShared));
   });
   if (attr != cudaSuccess) return int(attr);
   CUtensorMap mw, ma;
-  if (!make_tma_2d_kmajor(&mw, W, true, N, K, kGuRows) || !make_tma_2d_kmajor(&ma, A, true, M, K, kGuSlots))
+  if (!make_tma_2d_kmajor(&mw, W, true, N, K, kGuRows) || !make_tma_2d_kmajor(&ma, A, true, M, K, NT))
     return int(cudaErrorInvalidValue);
   GuParams p{};
   p.a_scale = a_scale;
@@ -432,7 +514,7 @@ static int launch_gu(const void* A, const float* a_scale, const void* W, const f
 int launch_gemv_umma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
                           int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream) {
   if (M < 1 || M > kGemvMaxM || (N + kGuRows - 1) / kGuRows > kMaxCounters) return int(cudaErrorInvalidValue);
-  if (!gu_scales_fit(N, K))
+  if (!gu_scales_fit(M, N, K))
     return launch_gemv_tma_a8w8(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
   if (M <= 8) return launch_gu<8>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
   if (M <= 16) return launch_gu<16>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
