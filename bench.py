@@ -219,6 +219,8 @@ def run_gpu(args):
     for (N, K), u in uses.items():
         n = len(wcopies[(N, K)])
         period = period * (n // u) // math.gcd(period, n // u)
+    if period > 64:
+        raise SystemExit(f"weight rotation needs {period} graph phases; choose a rotation with a shorter period")
 
     stream = torch.cuda.Stream(device=dev)
     n_calls = len(calls)
@@ -482,11 +484,254 @@ def cpu_baseline(workload, budget_s=20.0):
                       f"{'; large-M calls timed on 64 rows and scaled by M/64' if workload in ('prefill', 'ladder') else ''}"}
 
 
+# --------------------------------------------------------------------------- bf16 small-N workload
+BF16_METRIC = "bf16 small-N GEMM µs/call, TFLOPS & HBM GB/s (cold weights) vs roofline"
+
+
+def bf16_calls():
+    """(M, N, K, out_fp32, nk_index, m_index) of the small-N BF16 workload."""
+    return [(M, N, K, f32, i, j) for i, (N, K, f32) in enumerate(inputs.BF16_NK) for j, M in enumerate(inputs.BF16_MS)]
+
+
+def _oracle_bf16_call(M, N, K, f32, i, j, wcache):
+    from oracle import gemm as ogemm
+    if (N, K) not in wcache:
+        wcache[(N, K)] = inputs.weight_bf16(N, K, inputs.decode_seed_w(i)).float().numpy()  # set-up, untimed
+    a = inputs.activation_bf16(M, K, inputs.decode_seed_a(i, j)).float().numpy()
+    t0 = time.perf_counter()
+    ogemm.gemm_bf16(a, wcache[(N, K)], out_fp32=f32)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_bf16(budget_s=20.0):
+    calls = bf16_calls()
+    order = list(np.random.default_rng(0).permutation(len(calls)))
+    wcache, spent, done = {}, 0.0, []
+    for c in order:
+        M, N, K, f32, i, j = calls[c]
+        m = min(M, 64)  # the oracle is row-separable: large-M calls are timed on 64 rows and scaled
+        dt = _oracle_bf16_call(m, N, K, f32, i, j, wcache)
+        spent += dt
+        done.append(dt * M / m)
+        if spent > budget_s:
+            break
+    return {"value": round(float(np.mean(done)) * 1e6, 1), "unit": "µs/call", "cores": _threads(), "kind": "oracle",
+            "sample": f"{len(done)} of {len(calls)} calls of the bf16_small_n workload (random order), float64 "
+                      "matmul; calls with M > 64 timed on 64 rows and scaled by M/64"}
+
+
+def run_gpu_bf16(args):
+    import torch
+    import torch.distributed as dist
+
+    import fp8_block_scaled_a8w8_b200 as fb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    fb.lib()
+    pk = peaks()
+    calls = bf16_calls()
+    n_calls = len(calls)
+    uses, maxm = {}, {}
+    for (M, N, K, f32, i, j) in calls:
+        uses[(N, K)] = uses.get((N, K), 0) + 1
+        maxm[(N, K)] = max(maxm.get((N, K), 0), M)
+    wcopies, bx, bo = {}, {}, {}
+    for (M, N, K, f32, i, j) in calls:
+        if (N, K) in wcopies:
+            continue
+        w = inputs.weight_bf16(N, K, inputs.decode_seed_w(i)).to(dev)
+        # one distinct copy per use within a step (each call reads cold weights); between two
+        # steps the large-M calls stream > 1 GB of activations, far above the 126 MB L2
+        wcopies[(N, K)] = [w] + [w.clone() for _ in range(uses[(N, K)] - 1)]
+        bx[(N, K)] = inputs.activation_bf16(maxm[(N, K)], K, inputs.decode_seed_a(i, 0)).to(dev)
+        bo[(N, K)] = torch.empty((maxm[(N, K)], N), dtype=torch.float32 if f32 else torch.bfloat16, device=dev)
+    xs = [bx[(N, K)][:M] for (M, N, K, *_r) in calls]
+    outs = [bo[(N, K)][:M] for (M, N, K, *_r) in calls]
+    workspace = torch.zeros(max(256, max(fb.workspace_bytes(fb.OP_BF16, M, N, K) for (M, N, K, *_r) in calls)),
+                            dtype=torch.uint8, device=dev)
+    cfgs = [fb.dispatch_lookup(fb.OP_BF16, M, N, K)[1] for (M, N, K, *_r) in calls]
+    period = 1
+    stream = torch.cuda.Stream(device=dev)
+
+    def step_launches(s, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        ctr = {}
+        for c, (M, N, K, f32, *_r) in enumerate(calls):
+            k = ctr.get((N, K), 0)
+            ctr[(N, K)] = k + 1
+            cp = wcopies[(N, K)]
+            fb.gemm_bf16(xs[c], cp[(s * uses[(N, K)] + k) % len(cp)], out_fp32=f32, out=outs[c], workspace=workspace,
+                         stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    events = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(period)]
+    graphs = []
+    fb.dispatch_reset_stats()
+    with torch.cuda.stream(stream):
+        for ph in range(period):
+            step_launches(ph)
+        stream.synchronize()
+        for ph in range(period):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step_launches(ph, events[ph])
+            graphs.append(g)
+    torch.cuda.synchronize()
+    census = fb.dispatch_stats(fb.OP_BF16)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            graphs[s % period].replay()
+    barrier()
+    clocks = ClockSampler(dev.index)
+    if rank == 0:
+        clocks.start()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    t_start.record(stream)
+    for s in range(args.steps):
+        with torch.cuda.stream(stream):
+            graphs[(args.warmup + s) % period].replay()
+    t_end.record(stream)
+    barrier()
+    clk = clocks.stop() if rank == 0 else None
+    step_ms = t_start.elapsed_time(t_end) / args.steps
+    t = torch.tensor([step_ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms = float(t.item())
+
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e_steps = min(args.e2e_steps, 5)
+        hx = [x.cpu().pin_memory() for x in xs]
+        hy = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+        dxb = {k: torch.empty_like(v) for k, v in bx.items()}
+        dx = [dxb[(N, K)][:M] for (M, N, K, *_r) in calls]
+        h2d = sum(x.numel() * x.element_size() for x in xs)
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+
+        def e2e_step(s):
+            with torch.cuda.stream(stream):
+                ctr = {}
+                for c, (M, N, K, f32, *_r) in enumerate(calls):
+                    dx[c].copy_(hx[c], non_blocking=True)
+                    k = ctr.get((N, K), 0)
+                    ctr[(N, K)] = k + 1
+                    cp = wcopies[(N, K)]
+                    fb.gemm_bf16(dx[c], cp[(s * uses[(N, K)] + k) % len(cp)], out_fp32=f32, out=outs[c],
+                                 workspace=workspace, stream=stream)
+                    hy[c].copy_(outs[c], non_blocking=True)
+        for s in range(2):
+            e2e_step(s)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(e2e_steps):
+            e2e_step(s)
+        e1.record(stream)
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": round(float(te.item()) * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "api": "fp8_block_scaled_a8w8_b200.gemm_bf16 (eager)"}
+
+    if rank == 0:
+        gemm_ms = float(np.mean([events[ph][0].elapsed_time(events[ph][1]) for ph in sorted(
+            {(args.warmup + s) % period for s in range(args.steps)})]))
+        tot_bytes = float(sum(bf16_bytes(M, N, K, f32) for (M, N, K, f32, *_r) in calls))
+        tot_flops = float(sum(2.0 * M * N * K for (M, N, K, *_r) in calls))
+        peak_tf = pk["bf16_tflops_sustained"]
+        t_hbm = tot_bytes / (pk["hbm_gbs"] * 1e9)
+        t_tc = tot_flops / (peak_tf * 1e12)
+        t_roof = sum(max(bf16_bytes(M, N, K, f32) / (pk["hbm_gbs"] * 1e9), 2.0 * M * N * K / (peak_tf * 1e12))
+                     for (M, N, K, f32, *_r) in calls)
+        if t_hbm >= t_tc:
+            ach = tot_bytes / (gemm_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(ach / pk["hbm_gbs"], 4),
+                    "peak_source": f"{pk['source']} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"}
+        else:
+            ach = tot_flops / (gemm_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak_tf, "unit": "TFLOP/s",
+                    "frac": round(ach / peak_tf, 4),
+                    "peak_source": f"{pk['source']} sustained bf16 cuBLAS (MEASURED_PEAKS.json bf16_tflops_sustained)"}
+        roof["traffic"] = None
+        roof["roofline_time_frac"] = round(t_roof / (gemm_ms * 1e-3), 4)
+        roof["kernel"] = "gemm_bf16: " + ", ".join(sorted(set(cfgs)))
+        roof["gemm_us_per_step"] = round(gemm_ms * 1000.0, 2)
+        detail = None
+        if args.detail:
+            detail = []
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for c, (M, N, K, f32, *_r) in enumerate(calls):
+                cp = wcopies[(N, K)]
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    with torch.cuda.graph(g, stream=stream):
+                        for r in range(20):
+                            fb.gemm_bf16(xs[c], cp[r % len(cp)], out_fp32=f32, out=outs[c], workspace=workspace,
+                                         stream=stream)
+                    ts = []
+                    for _ in range(5):
+                        e0.record(stream)
+                        g.replay()
+                        e1.record(stream)
+                        e1.synchronize()
+                        ts.append(e0.elapsed_time(e1) * 1000.0 / 20)
+                del g
+                us = sorted(ts)[len(ts) // 2]
+                by, fl = bf16_bytes(M, N, K, f32), 2.0 * M * N * K
+                roof_us = max(by / (pk["hbm_gbs"] * 1e3), fl / (peak_tf * 1e6))
+                detail.append({"M": M, "N": N, "K": K, "out": "f32" if f32 else "bf16", "cfg": cfgs[c],
+                               "us": round(us, 3), "GBps": round(by / us / 1e3, 1), "TFLOPS": round(fl / us / 1e6, 2),
+                               "roofline_frac": round(roof_us / us, 3)})
+        cpu = cpu_baseline_bf16() if (args.cpu_baseline and world == 1) else None
+        line = {
+            "metric": BF16_METRIC, "value": round(step_ms * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x bf16 -> f32",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no dataset)",
+            "config": {"workload": "bf16_small_n", "description": inputs.WORKLOADS["bf16_small_n"],
+                       "calls_per_step": n_calls, "weight_rotation_mib": ROTATE_BYTES >> 20,
+                       "l2": "one weight copy per use within a step; > 1 GB of activations streamed per step (L2 126 MB)",
+                       "parallelism": f"replicas x{world}", "timing": "CUDA graphs replayed, CUDA events, max over ranks"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": n_calls * args.steps,
+            "clocks": clk, "dispatch": {**census, "table_hash": fb.dispatch_table_hash()}, "detail": detail,
+        }
+        print(json.dumps(line), flush=True)
+    for g in graphs:
+        del g
+    graphs.clear()
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if world > 1 and rank != 0:
         return
+    if args.workload == "bf16_small_n":
+        return run_reference_bf16(args, world)
     calls = workload_calls(args.workload)
     wcache = {}
     for s in range(args.warmup):
@@ -509,6 +754,29 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_bf16(args, world):
+    calls = bf16_calls()
+    wcache = {}
+    for s in range(args.warmup):
+        M, N, K, f32, i, j = calls[s % len(calls)]
+        _oracle_bf16_call(min(M, 64), N, K, f32, i, j, wcache)
+    times = []
+    for s in range(args.steps):
+        M, N, K, f32, i, j = calls[(args.warmup + s) % len(calls)]
+        m = min(M, 64)
+        times.append(_oracle_bf16_call(m, N, K, f32, i, j, wcache) * M / m)
+    us = float(np.mean(times)) * 1e6
+    line = {"impl": "reference", "metric": BF16_METRIC, "value": round(us, 1), "unit": "µs/call", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1000.0, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "bf16_small_n", "description": inputs.WORKLOADS["bf16_small_n"]},
+            "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": _threads(), "kind": "oracle",
+                             "sample": "one call per step, cycling through the bf16_small_n calls; M > 64 timed on "
+                                       "64 rows and scaled"},
+            "e2e": {"value": round(us, 1), "unit": "µs/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -526,6 +794,8 @@ def main():
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "bf16_small_n" and not args.shape:
+        run_gpu_bf16(args)
     else:
         run_gpu(args)
 
