@@ -30,15 +30,15 @@ static const KernelConfig kConfigs[] = {
     {"a8w8_gemv_d4", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemv, 0, 1, 4},
     {"a8w8_gemv_tma", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemvTma, 0, 1, 0},
     {"a8w8_gemv_umma", FP8BS_OP_A8W8_BLOCKSCALE, kPathGemvUmma, 0, 1, 0},
-    {"a8w8_tc_bn128", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 128, 1, 0},
-    {"a8w8_tc_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 256, 1, 0},
+    {"a8w8_tc_bn128", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 128, 0, 0},
+    {"a8w8_tc_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 256, 0, 0},
     {"bf16_gemv_d2", FP8BS_OP_BF16, kPathGemv, 0, 1, 2},
     {"bf16_gemv_d4", FP8BS_OP_BF16, kPathGemv, 0, 1, 4},
-    {"bf16_tc_bn32", FP8BS_OP_BF16, kPathTc, 32, 1, 0},
-    {"bf16_tc_bn64", FP8BS_OP_BF16, kPathTc, 64, 1, 0},
-    {"bf16_tc_bn128", FP8BS_OP_BF16, kPathTc, 128, 1, 0},
-    {"bf16_tc_bn192", FP8BS_OP_BF16, kPathTc, 192, 1, 0},
-    {"bf16_tc_bn256", FP8BS_OP_BF16, kPathTc, 256, 1, 0},
+    {"bf16_tc_bn32", FP8BS_OP_BF16, kPathTc, 32, 0, 0},
+    {"bf16_tc_bn64", FP8BS_OP_BF16, kPathTc, 64, 0, 0},
+    {"bf16_tc_bn128", FP8BS_OP_BF16, kPathTc, 128, 0, 0},
+    {"bf16_tc_bn192", FP8BS_OP_BF16, kPathTc, 192, 0, 0},
+    {"bf16_tc_bn256", FP8BS_OP_BF16, kPathTc, 256, 0, 0},
 };
 static constexpr int kNumConfigs = sizeof(kConfigs) / sizeof(kConfigs[0]);
 
@@ -60,24 +60,43 @@ const KernelConfig* const* list_configs(int op, int* count) {
   return lists[op];
 }
 
+// Tensor-core tile width: the widest candidate (fewest re-reads of A) whose output tiles
+// still give at least half of the SMs a tile; if none does, the narrowest (the kernel then
+// also splits K).
+static int pick_bn(int64_t M, int64_t N, const int* cands, int n) {
+  const int64_t m_tiles = (M + 127) / 128;
+  const int64_t half_sms = (int64_t(device_sm_count()) + 1) / 2;
+  for (int i = 0; i < n; ++i)
+    if (m_tiles * ((N + cands[i] - 1) / cands[i]) >= half_sms) return cands[i];
+  return cands[n - 1];
+}
+
 const KernelConfig* default_config(int op, int64_t M, int64_t N, int64_t K) {
   (void)K;
+  char nm[32];
   if (op == FP8BS_OP_A8W8_BLOCKSCALE) {
     if (M <= kGemvMaxM) return find_config(op, "a8w8_gemv_umma");
-    if (N % 256 == 0) return find_config(op, "a8w8_tc_bn256");
-    return find_config(op, "a8w8_tc_bn128");
-  }
-  if (M <= kGemvMaxM) return find_config(op, M <= 16 ? "bf16_gemv_d4" : "bf16_gemv_d2");
-  if (N <= 256 && (N == 32 || N == 64 || N == 128 || N == 192 || N == 256)) {
-    char nm[32];
-    std::snprintf(nm, sizeof nm, "bf16_tc_bn%d", int(N));
+    static const int fp8_bn[] = {256, 128};
+    const int bn = (N % 256 == 0) ? pick_bn(M, N, fp8_bn, 2) : 128;
+    std::snprintf(nm, sizeof nm, "a8w8_tc_bn%d", bn);
     return find_config(op, nm);
   }
-  if (N % 256 == 0) return find_config(op, "bf16_tc_bn256");
-  if (N % 192 == 0) return find_config(op, "bf16_tc_bn192");
-  if (N % 128 == 0) return find_config(op, "bf16_tc_bn128");
-  if (N % 64 == 0) return find_config(op, "bf16_tc_bn64");
-  return find_config(op, "bf16_tc_bn32");
+  if (M <= kGemvMaxM) return find_config(op, M <= 16 ? "bf16_gemv_d4" : "bf16_gemv_d2");
+  // widest first among the widths that tile N without a ragged last tile, then narrower
+  static const int all_bn[] = {256, 192, 128, 64, 32};
+  int cands[5], n = 0;
+  for (int b : all_bn)
+    if (b <= N && N % b == 0) cands[n++] = b;
+  if (n == 0) cands[n++] = 32;
+  if (N < 256 && N % 32 == 0 && N != cands[0]) {  // a single tile as wide as N comes first
+    for (int i = n; i > 0; --i) cands[i] = cands[i - 1];
+    cands[0] = int(N);
+    ++n;
+  }
+  int bn = pick_bn(M, N, cands, n);
+  if (bn != 32 && bn != 64 && bn != 128 && bn != 192 && bn != 256) bn = 32;
+  std::snprintf(nm, sizeof nm, "bf16_tc_bn%d", bn);
+  return find_config(op, nm);
 }
 
 // ------------------------------------------------------------ table + census

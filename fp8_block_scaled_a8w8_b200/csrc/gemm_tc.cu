@@ -70,7 +70,12 @@ struct TcParams {
   int kblocks;           // K blocks of 128 bytes
   int m_tiles, n_tiles;
   int out_fp32;
+  int splits;            // K splits per output tile (1 = none)
+  float* part;           // splits > 1: [tiles * splits][kBM][BN] float32 partial tiles
+  unsigned* counter;     // splits > 1: [tiles] arrival counters (left at zero)
 };
+
+__device__ __forceinline__ void tc_epilogue_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_ld_chunk16(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -119,7 +124,62 @@ __device__ __forceinline__ void store_row_chunk(const TcParams& p, int row, int 
   }
 }
 
-template <bool kFp8, int BN>
+// Split K: every split stores its float32 partial tile; after all epilogue threads have
+// stored, one thread counts the split in (gpu-scope acq_rel atomic after the epilogue
+// barrier), and the split that arrives last sums the tile's partials in split order -- a
+// fixed order, so results are bit-reproducible -- rounds once and resets the counter.
+template <int kChunk>
+__device__ __forceinline__ void tc_store_partial(const TcParams& p, float* dst, int row, const float* v) {
+  if (row >= p.M) return;
+#pragma unroll
+  for (int j = 0; j < kChunk; j += 4) __stcg(reinterpret_cast<float4*>(dst + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+}
+
+template <int BN, int kHalf, int kChunk>
+__device__ __forceinline__ void tc_splitk_finish(const TcParams& p, int tile, int row_in_tile, int row, int h,
+                                                 int col0, volatile unsigned* s_old, volatile int* abort_flag) {
+  tc_epilogue_bar();  // every epilogue thread's partial stores precede the release below
+  // after a timed-out wait nothing is published (the status word reports it; the caller
+  // re-zeroes the workspace before reusing it)
+  if (threadIdx.x == 128) *s_old = *abort_flag ? ~0u : atom_add_acq_rel_gpu(p.counter + tile, 1u);
+  tc_epilogue_bar();
+  if (*s_old != unsigned(p.splits - 1)) return;
+  if (row < p.M) {
+#pragma unroll 1
+    for (int c = 0; c < kHalf / kChunk; ++c) {
+      float sum[kChunk];
+#pragma unroll
+      for (int j = 0; j < kChunk; ++j) sum[j] = 0.f;
+      constexpr int kPar = kChunk >= 32 ? 2 : 4;  // splits' loads in flight (64 floats)
+#pragma unroll 1
+      for (int sp = 0; sp < p.splits; sp += kPar) {
+        float v[kPar][kChunk];
+#pragma unroll
+        for (int k = 0; k < kPar; ++k) {
+          const float* src = p.part + ((int64_t(tile) * p.splits + sp + k) * kBM + row_in_tile) * BN + h * kHalf + c * kChunk;
+#pragma unroll
+          for (int j = 0; j < kChunk; j += 4) {
+            const float4 f = sp + k < p.splits ? __ldcg(reinterpret_cast<const float4*>(src + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[k][j] = f.x;
+            v[k][j + 1] = f.y;
+            v[k][j + 2] = f.z;
+            v[k][j + 3] = f.w;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kPar; ++k)
+#pragma unroll
+          for (int j = 0; j < kChunk; ++j) sum[j] += v[k][j];
+      }
+      store_row_chunk<kChunk>(p, row, col0 + c * kChunk, sum);
+    }
+  }
+  if (threadIdx.x == 128) p.counter[tile] = 0u;
+}
+
+// kSplitK: instantiated with split-K support; without it the kernel is exactly the
+// one-split kernel (no split bookkeeping in the register budget of the hot loop).
+template <bool kFp8, int BN, bool kSplitK>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcParams p) {
   using C = TcCfg<kFp8, BN>;
@@ -132,6 +192,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // bars: full[S], empty[S], tmem_full[2], tmem_empty[2], drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile unsigned* s_old = reinterpret_cast<volatile unsigned*>(tmem_slot + 2);  // split-K arrival
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -166,7 +227,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   pdl_wait();  // the previous kernel's results are visible from here
   const uint32_t tmem_base = *tmem_slot;
 
-  const int tiles_total = p.m_tiles * p.n_tiles;
+  // work items: (output tile, K split); item -> tile = item / splits, K blocks [kb0, kb1)
+  const int splits = kSplitK ? p.splits : 1;
+  const int items = p.m_tiles * p.n_tiles * splits;
   const int KB = p.kblocks;
   const int G = p.K / 128;  // scale groups (a8w8)
 
@@ -179,9 +242,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int last_it[8];
       for (int s = 0; s < S; ++s) last_it[s] = -1;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles_total && ok; tile += gridDim.x) {
+      for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+        const int tile = item / splits, sp = item - tile * splits;
+        const int kb0 = KB * sp / splits, kb1 = KB * (sp + 1) / splits;
         const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % S;
           if (!mbar_wait_bounded(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, &g_status)) {
             ok = false;
@@ -214,7 +279,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int it = 0, acc_it = 0, tile_it = 0;
       bool ok = true;
       bool issued = false;
-      for (int tile = blockIdx.x; tile < tiles_total && ok; tile += gridDim.x, ++tile_it) {
+      for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++tile_it) {
+        const int sp = item % splits;
+        const int kb0 = KB * sp / splits, kb1 = KB * (sp + 1) / splits;
         uint32_t d_tmem = 0;
         int tb = tile_it & 1;
         if (!kFp8) {
@@ -222,7 +289,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_fence_after();
           d_tmem = tmem_base + uint32_t(tb * BN);
         }
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % S;
           if (!mbar_wait_bounded(full_bar(s), (it / S) & 1, abort_flag, &g_status)) {
             ok = false;
@@ -244,7 +311,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint64_t bdesc = sw128_kmajor_desc(a_addr + C::kABytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t acc = kFp8 ? (kk > 0) : (kb > 0 || kk > 0);
+            const uint32_t acc = kFp8 ? (kk > 0) : (kb > kb0 || kk > 0);
             if (kFp8)
               umma_f8f6f4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, C::kIdesc, acc);
             else
@@ -280,7 +347,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lane_addr = tmem_base + (uint32_t(32 * q) << 16);
     int acc_it = 0, tile_it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles_total && ok; tile += gridDim.x, ++tile_it) {
+    // With split K every epilogue warp goes through every item, also after a timed-out wait
+    // (then without touching TMEM or memory), so the epilogue barriers of the split-K
+    // finish always see all eight warps.
+    for (int item = blockIdx.x; item < items && (kSplitK || ok); item += gridDim.x, ++tile_it) {
+      const int tile = item / splits, sp = item - tile * splits;
+      const int kb0 = KB * sp / splits, kb1 = KB * (sp + 1) / splits;
       const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
       const int row = tm * kBM + row_in_tile;
       const int col0 = tn * BN + h * C::kHalfCols;
@@ -293,21 +365,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const float* asrow = p.a_scale + int64_t(row < p.M ? row : 0) * G;
         const bool row_ok = row < p.M;
         // a_scale of this row, four groups ahead (L1 hits after the first touch of the row)
-        float sa0 = row_ok ? __ldg(asrow + 0) : 0.f;
-        float sa1 = (row_ok && KB > 1) ? __ldg(asrow + 1) : 0.f;
-        float sa2 = (row_ok && KB > 2) ? __ldg(asrow + 2) : 0.f;
-        float sa3 = (row_ok && KB > 3) ? __ldg(asrow + 3) : 0.f;
-        float sw0 = nb_ok ? __ldg(p.w_scale + int64_t(nbw) * G) : 0.f;
-        for (int kb = 0; kb < KB; ++kb) {
+        float sa0 = row_ok ? __ldg(asrow + kb0) : 0.f;
+        float sa1 = (row_ok && kb0 + 1 < kb1) ? __ldg(asrow + kb0 + 1) : 0.f;
+        float sa2 = (row_ok && kb0 + 2 < kb1) ? __ldg(asrow + kb0 + 2) : 0.f;
+        float sa3 = (row_ok && kb0 + 3 < kb1) ? __ldg(asrow + kb0 + 3) : 0.f;
+        float sw0 = nb_ok ? __ldg(p.w_scale + int64_t(nbw) * G + kb0) : 0.f;
+        for (int kb = kb0; kb < kb1; ++kb) {
           const float sc = sa0 * sw0;
           sa0 = sa1;
           sa1 = sa2;
           sa2 = sa3;
-          sa3 = (row_ok && kb + 4 < KB) ? __ldg(asrow + kb + 4) : 0.f;
-          sw0 = (nb_ok && kb + 1 < KB) ? __ldg(p.w_scale + int64_t(nbw) * G + kb + 1) : 0.f;
+          sa3 = (row_ok && kb + 4 < kb1) ? __ldg(asrow + kb + 4) : 0.f;
+          sw0 = (nb_ok && kb + 1 < kb1) ? __ldg(p.w_scale + int64_t(nbw) * G + kb + 1) : 0.f;
           const int b = acc_it & 1;
+          if (kSplitK && !ok) continue;
           if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (acc_it >> 1) & 1, abort_flag, &g_status))) {
             ok = false;
+            if (kSplitK) continue;
             break;
           }
           tc_fence_after();
@@ -341,28 +415,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           ++acc_it;
         }
-        if (!ok) break;
+        if (!kSplitK) {
+          if (!ok) break;
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) store_row_chunk<C::kChunk>(p, row, col0 + c * C::kChunk, acc + c * C::kChunk);
+          for (int c = 0; c < C::kChunks; ++c) store_row_chunk<C::kChunk>(p, row, col0 + c * C::kChunk, acc + c * C::kChunk);
+        } else {
+          if (ok) {
+            float* part_row = p.part + (int64_t(item) * kBM + row_in_tile) * BN + h * C::kHalfCols;
+#pragma unroll
+            for (int c = 0; c < C::kChunks; ++c)
+              tc_store_partial<C::kChunk>(p, part_row + c * C::kChunk, row, acc + c * C::kChunk);
+          }
+          tc_splitk_finish<BN, C::kHalfCols, C::kChunk>(p, tile, row_in_tile, row, h, col0, s_old, abort_flag);
+        }
       } else {
         const int b = tile_it & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (tile_it >> 1) & 1, abort_flag, &g_status)))
-          break;
-        tc_fence_after();
-        const uint32_t t_addr = lane_addr + uint32_t(b * BN + h * C::kHalfCols);
+        if (ok && !__all_sync(0xffffffffu, mbar_wait_bounded(tfull_bar(b), (tile_it >> 1) & 1, abort_flag, &g_status)))
+          ok = false;
+        if (!ok && !kSplitK) break;
+        if (ok) {
+          tc_fence_after();
+          const uint32_t t_addr = lane_addr + uint32_t(b * BN + h * C::kHalfCols);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) {
-          uint32_t r[32];
-          tmem_ld<C::kChunk>(t_addr + c * C::kChunk, r);
-          tmem_ld_wait();
-          float v[C::kChunk];
+          for (int c = 0; c < C::kChunks; ++c) {
+            uint32_t r[32];
+            tmem_ld<C::kChunk>(t_addr + c * C::kChunk, r);
+            tmem_ld_wait();
+            float v[C::kChunk];
 #pragma unroll
-          for (int j = 0; j < C::kChunk; ++j) v[j] = __uint_as_float(r[j]);
-          store_row_chunk<C::kChunk>(p, row, col0 + c * C::kChunk, v);
+            for (int j = 0; j < C::kChunk; ++j) v[j] = __uint_as_float(r[j]);
+            if (!kSplitK)
+              store_row_chunk<C::kChunk>(p, row, col0 + c * C::kChunk, v);
+            else
+              tc_store_partial<C::kChunk>(
+                  p, p.part + (int64_t(item) * kBM + row_in_tile) * BN + h * C::kHalfCols + c * C::kChunk, row, v);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(b));
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(b));
+        if (kSplitK) tc_splitk_finish<BN, C::kHalfCols, C::kChunk>(p, tile, row_in_tile, row, h, col0, s_old, abort_flag);
       }
     }
   }
@@ -376,25 +468,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-template <bool kFp8, int BN>
-static int launch_tc_t(const void* A, const void* W, const TcParams& prm, void* stream) {
+template <bool kFp8, int BN, bool kSplitK>
+static int launch_tc_split(const void* A, const void* W, const TcParams& prm, void* stream) {
   using C = TcCfg<kFp8, BN>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_tc_kernel<kFp8, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    attr_err = cudaFuncSetAttribute(gemm_tc_kernel<kFp8, BN, kSplitK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     int(C::kSmemBytes));
   });
   if (attr_err != cudaSuccess) return int(attr_err);
   CUtensorMap ma, mb;
   if (!make_tma_2d_kmajor(&ma, A, kFp8, prm.M, prm.K, kBM) || !make_tma_2d_kmajor(&mb, W, kFp8, prm.N, prm.K, BN))
     return int(cudaErrorInvalidValue);
-  const int tiles = prm.m_tiles * prm.n_tiles;
+  const int tiles = prm.m_tiles * prm.n_tiles * prm.splits;
   const int grid = std::min(tiles, device_sm_count());
-  return launch_kernel(gemm_tc_kernel<kFp8, BN>, dim3(grid), dim3(kTcThreads), C::kSmemBytes, stream, ma, mb, prm);
+  return launch_kernel(gemm_tc_kernel<kFp8, BN, kSplitK>, dim3(grid), dim3(kTcThreads), C::kSmemBytes, stream, ma, mb,
+                       prm);
 }
 
-size_t tc_workspace_bytes(int, int64_t, int64_t, int64_t, const KernelConfig&) { return 0; }
+template <bool kFp8, int BN>
+static int launch_tc_t(const void* A, const void* W, const TcParams& prm, void* stream) {
+  return prm.splits > 1 ? launch_tc_split<kFp8, BN, true>(A, W, prm, stream)
+                        : launch_tc_split<kFp8, BN, false>(A, W, prm, stream);
+}
+
+// K splits for a shape: the configuration's split_k if set, else automatic -- split only
+// when the output tiles leave most SMs idle, into enough splits to fill about one wave, at
+// most 8 and at least two K blocks per split (the partial tiles cost 8 bytes of traffic per
+// output element per split).
+static int tc_splits(const KernelConfig& cfg, int64_t M, int64_t N, int64_t K, bool fp8) {
+  const int64_t kb = fp8 ? K / 128 : K / 64;
+  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + cfg.bn - 1) / cfg.bn);
+  int64_t sp = cfg.split_k;
+  if (sp <= 0) {
+    const int64_t sms = device_sm_count();
+    sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({(sms + tiles - 1) / tiles, kb / 2, 8});
+  }
+  sp = std::max<int64_t>(1, std::min(sp, kb));
+  if (sp > 1 && tiles > kMaxCounters) sp = 1;
+  return int(sp);
+}
+
+size_t tc_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, const KernelConfig& cfg) {
+  const bool fp8 = op == FP8BS_OP_A8W8_BLOCKSCALE;
+  const int sp = tc_splits(cfg, M, N, K, fp8);
+  if (sp == 1) return 0;
+  const int64_t tiles = ((M + kBM - 1) / kBM) * ((N + cfg.bn - 1) / cfg.bn);
+  return kCounterBytes + size_t(tiles) * sp * kBM * cfg.bn * sizeof(float);
+}
 
 static TcParams make_params(const float* a_scale, const float* w_scale, void* out, int64_t M, int64_t N, int64_t K,
                             int bn, bool fp8, int out_fp32) {
@@ -409,12 +531,24 @@ static TcParams make_params(const float* a_scale, const float* w_scale, void* ou
   p.m_tiles = int((M + kBM - 1) / kBM);
   p.n_tiles = int((N + bn - 1) / bn);
   p.out_fp32 = out_fp32;
+  p.splits = 1;
   return p;
 }
 
+static int set_splits(TcParams& p, const KernelConfig& cfg, bool fp8, void* ws) {
+  p.splits = tc_splits(cfg, p.M, p.N, p.K, fp8);
+  if (p.splits > 1) {
+    if (!ws) return int(cudaErrorInvalidValue);
+    p.counter = static_cast<unsigned*>(ws);
+    p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
+  }
+  return 0;
+}
+
 int launch_tc_a8w8(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W,
-                   const float* w_scale, void* out, int64_t M, int64_t N, int64_t K, void*, void* stream) {
-  const TcParams p = make_params(a_scale, w_scale, out, M, N, K, cfg.bn, true, 0);
+                   const float* w_scale, void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream) {
+  TcParams p = make_params(a_scale, w_scale, out, M, N, K, cfg.bn, true, 0);
+  if (const int e = set_splits(p, cfg, true, ws)) return e;
   switch (cfg.bn) {
     case 128: return launch_tc_t<true, 128>(A, W, p, stream);
     case 256: return launch_tc_t<true, 256>(A, W, p, stream);
@@ -423,8 +557,9 @@ int launch_tc_a8w8(const KernelConfig& cfg, const void* A, const float* a_scale,
 }
 
 int launch_tc_bf16(const KernelConfig& cfg, const void* A, const void* W, void* out, int out_fp32, int64_t M,
-                   int64_t N, int64_t K, void*, void* stream) {
-  const TcParams p = make_params(nullptr, nullptr, out, M, N, K, cfg.bn, false, out_fp32);
+                   int64_t N, int64_t K, void* ws, void* stream) {
+  TcParams p = make_params(nullptr, nullptr, out, M, N, K, cfg.bn, false, out_fp32);
+  if (const int e = set_splits(p, cfg, false, ws)) return e;
   switch (cfg.bn) {
     case 32: return launch_tc_t<false, 32>(A, W, p, stream);
     case 64: return launch_tc_t<false, 64>(A, W, p, stream);

@@ -209,17 +209,35 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs p) {
               for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) sum[nb][i] = 0.f;
-              for (int64_t ww = wf; ww <= wl; ++ww) {
-                const int ft = int((U * ww / Wn) / G);
-                const int sl = 2 * int(ww) + (t == ft ? 0 : 1);
-                float* src = p.part + int64_t(sl) * (NB * 4 * 32);
+              // contributors' partials in warp order (a fixed order), kRB warps' loads in flight
+              constexpr int kRB = NB == 1 ? 8 : NB == 2 ? 4 : 2;
+              for (int64_t w0 = wf; w0 <= wl; w0 += kRB) {
+                float v[kRB][NB][4];
+                float* srcs[kRB];
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb)
+                for (int j = 0; j < kRB; ++j) {
+                  const int64_t ww = w0 + j;
+                  const int ft = int((U * ww / Wn) / G);
+                  srcs[j] = p.part + int64_t(2 * ww + (t == ft ? 0 : 1)) * (NB * 4 * 32);
 #pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    sum[nb][i] += __ldcg(src + (nb * 4 + i) * 32 + lane);
-                    __stcg(src + (nb * 4 + i) * 32 + lane, 0.f);  // leave the workspace zero-filled
+                  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) v[j][nb][i] = ww <= wl ? __ldcg(srcs[j] + (nb * 4 + i) * 32 + lane) : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < kRB; ++j) {
+#pragma unroll
+                  for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) sum[nb][i] += v[j][nb][i];
+                  if (w0 + j <= wl) {
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                      for (int i = 0; i < 4; ++i)
+                        __stcg(srcs[j] + (nb * 4 + i) * 32 + lane, 0.f);  // leave the workspace zero-filled
                   }
+                }
               }
               store_out<kFp8, NB>(p, t, lane, sum);
               if (lane == 0) p.counter[t] = 0u;
@@ -255,10 +273,14 @@ static int occupancy() {
 
 static int gemv_nb(int64_t M) { return int((M + 7) / 8); }
 
-// Warps the kernel runs with: one full wave of co-resident CTAs, never more warps than units.
+// Warps the kernel runs with: one full wave of co-resident CTAs, but at least
+// kMinUnitsPerWarp units per warp. (A small weight spread one unit per warp leaves every
+// 16-row tile with dozens of contributors, and the finishing warp's sum over them, not
+// the weight stream, sets the time.)
+constexpr int64_t kMinUnitsPerWarp = 8;
 static int64_t gemv_active_warps(int64_t units, int occ) {
   const int64_t warps = int64_t(device_sm_count()) * occ * kGemvWarps;
-  return std::min(warps, units);
+  return std::max<int64_t>(1, std::min(warps, units / kMinUnitsPerWarp));
 }
 
 template <bool kFp8, int NB>

@@ -27,7 +27,7 @@ struct KernelConfig {
   int op;           // FP8BS_OP_*
   int path;         // Path
   int bn;           // tensor-core path: N tile (columns of W per CTA)
-  int split_k;      // tensor-core path: K splits (1 = none)
+  int split_k;      // tensor-core path: K splits (0 = automatic from the tile count, 1 = none)
   int gemv_depth;   // weight-streaming path: units in flight per warp
 };
 

@@ -110,7 +110,8 @@ def test_census_counts_and_dedup():
     by_m = {r["M"]: r for r in recs}
     assert by_m[3]["padded_M"] == 4 and by_m[3]["count"] == 3 and by_m[3]["hit"]
     assert by_m[6016]["padded_M"] == 8192
-    assert by_m[40]["hit"] is False and by_m[40]["cfg"] == "a8w8_tc_bn256"
+    # a miss runs the default: 1 x 4 tiles of 256 columns would leave most SMs idle, so 128
+    assert by_m[40]["hit"] is False and by_m[40]["cfg"] == "a8w8_tc_bn128"
     fb.dispatch_reset_stats()
     assert fb.dispatch_stats(fb.OP_A8W8_BLOCKSCALE)["hits"] == 0
 
