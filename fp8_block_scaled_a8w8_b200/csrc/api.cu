@@ -59,7 +59,8 @@ static size_t op_workspace(int op, int64_t M, int64_t N, int64_t K, const Kernel
   switch (cfg.path) {
     case kPathGemv: return gemv_workspace_bytes(op, M, N, K, cfg);
     case kPathGemvTma: return gemv_tma_workspace_bytes(M, N, K);
-    case kPathGemvUmma: return gemv_umma_workspace_bytes(M, N, K);
+    case kPathGemvUmma:
+      return op == FP8BS_OP_BF16 ? gemv_umma_bf16_workspace_bytes(M, N, K) : gemv_umma_workspace_bytes(M, N, K);
     default: return tc_workspace_bytes(op, M, N, K, cfg);
   }
 }
@@ -195,6 +196,8 @@ FP8BS_API fp8bs_status fp8bs_gemm_bf16(const void* A_bf16, const void* W_bf16, v
   int e;
   if (cfg->path == kPathGemv)
     e = launch_gemv_bf16(*cfg, A_bf16, W_bf16, out, out_is_fp32, M, N, K, workspace, stream);
+  else if (cfg->path == kPathGemvUmma)
+    e = launch_gemv_umma_bf16(A_bf16, W_bf16, out, out_is_fp32, M, N, K, workspace, stream);
   else
     e = launch_tc_bf16(*cfg, A_bf16, W_bf16, out, out_is_fp32, M, N, K, workspace, stream);
   return from_cuda(e);

@@ -34,6 +34,7 @@ static const KernelConfig kConfigs[] = {
     {"a8w8_tc_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 256, 0, 0},
     {"bf16_gemv_d2", FP8BS_OP_BF16, kPathGemv, 0, 1, 2},
     {"bf16_gemv_d4", FP8BS_OP_BF16, kPathGemv, 0, 1, 4},
+    {"bf16_gemv_umma", FP8BS_OP_BF16, kPathGemvUmma, 0, 1, 0},
     {"bf16_tc_bn32", FP8BS_OP_BF16, kPathTc, 32, 0, 0},
     {"bf16_tc_bn64", FP8BS_OP_BF16, kPathTc, 64, 0, 0},
     {"bf16_tc_bn128", FP8BS_OP_BF16, kPathTc, 128, 0, 0},
@@ -81,7 +82,7 @@ const KernelConfig* default_config(int op, int64_t M, int64_t N, int64_t K) {
     std::snprintf(nm, sizeof nm, "a8w8_tc_bn%d", bn);
     return find_config(op, nm);
   }
-  if (M <= kGemvMaxM) return find_config(op, M <= 16 ? "bf16_gemv_d4" : "bf16_gemv_d2");
+  if (M <= kGemvMaxM) return find_config(op, "bf16_gemv_umma");
   // widest first among the widths that tile N without a ragged last tile, then narrower
   static const int all_bn[] = {256, 192, 128, 64, 32};
   int cands[5], n = 0;

@@ -84,17 +84,29 @@ static_assert(kGuCtasPerSm * (kGuSmemBytes + 1024) <= 233472, "two CTAs must fit
 static_assert(kGuCtasPerSm * kGuTmemCols <= 512, "two CTAs must fit an SM's TMEM");
 static_assert(kGuPrefetch <= kGuStages, "prefetch within the ring");
 constexpr uint32_t kGuIdesc = make_idesc(kFmtE4M3, kFmtE4M3, kGuRows, kGuSlots);
+constexpr uint32_t kGuIdescBf16 = make_idesc(kFmtBF16, kFmtBF16, kGuRows, kGuSlots);
+// A CTA takes at least this many units: a small weight spread over every SM would leave
+// each block with dozens of split-K contributors to sum.
+constexpr int64_t kGuMinUnitsPerCta = 8;
 
 struct GuParams {
   const float* a_scale;  // [M, G]
   const float* w_scale;  // [nblk, G]
-  __nv_bfloat16* out;    // [M, N]
+  void* out;             // [M, N] bf16 (or float32 when out_fp32)
   int M, N, G, nblk;
   int n_ctas;
   int static_w;          // W / w_scale are not written by any kernel still in flight
   float* part;           // [2 * n_ctas][kGuSlots][kGuRows]
   unsigned* counter;     // [nblk]
+  int out_fp32;          // bf16 GEMM only
 };
+
+__device__ __forceinline__ void gu_put(const GuParams& p, int64_t idx, float v) {
+  if (p.out_fp32)
+    static_cast<float*>(p.out)[idx] = v;
+  else
+    static_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+}
 
 __device__ __forceinline__ int64_t gu_cta_of_unit(int64_t u, int64_t U, int64_t C) { return ((u + 1) * C - 1) / U; }
 
@@ -158,14 +170,16 @@ __device__ __forceinline__ void gu_finish_block(const GuParams& p, int b, unsign
 #pragma unroll
     for (int j = 0; j < kE; ++j) {
       const int t = t0 + 2 * j;
-      if (t < p.M) p.out[int64_t(t) * p.N + n] = __float2bfloat16_rn(sum[j]);
+      if (t < p.M) gu_put(p, int64_t(t) * p.N + n, sum[j]);
     }
   }
   if (tid == 0) p.counter[b] = 0u;
 }
 
 // NT: token columns the epilogue reads per unit (8, 16 or 32 >= M).
-template <int NT>
+// kBf16: the bf16 GEMM (out = A W^T): a unit is 128 weight rows x 64 bf16 columns (the
+// same 128-byte rows), kind::f16 products, no scales.
+template <int NT, bool kBf16>
 __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
     gemv_umma_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmA, const GuParams p) {
   constexpr int S = kGuStages;
@@ -173,6 +187,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
   // The token box has NT rows (rows past M read as zero); MMA column n depends only on
   // token row n, so slots NT..31 may hold anything: their columns are never read.
   constexpr uint32_t kTx = kGuWBytes + NT * 128;
+  constexpr int kX = kBf16 ? 64 : 128;  // TMA x step per unit, in elements (128 bytes)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(S) * kGuStageBytes);  // full[S] empty[S] tfull[B] tempty[B] drain
@@ -243,13 +258,13 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (p.static_w) gu_order_bar_sync();  // the epilogue's w_scale requests go out first
+    if (!kBf16 && p.static_w) gu_order_bar_sync();  // the epilogue's w_scale requests go out first
     if (lane == 0) {
       int last_it[kGuStages];
       for (int s = 0; s < S; ++s) last_it[s] = -1;
       int b = first_blk, g = int(u0 - int64_t(first_blk) * G);
       int it = 0;
-      if (p.static_w) {
+      if (!kBf16 && p.static_w) {
         // The weights are not produced by an earlier kernel: fetch the first ring's worth
         // of weight boxes before waiting for the previous kernel, overlapping its tail.
         const int pre = n_units < kGuPrefetch ? n_units : kGuPrefetch;
@@ -257,7 +272,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
         for (int j = 0; j < pre; ++j) {
           const uint32_t dst = smem_u32(smem + size_t(j) * kGuStageBytes);
           mbar_arrive_expect_tx(full_bar(j), kTx);
-          tma_load_2d(dst, &tmW, full_bar(j), pg * 128, pb * kGuRows);
+          tma_load_2d(dst, &tmW, full_bar(j), pg * kX, pb * kGuRows);
           if (++pg == G) {
             pg = 0;
             ++pb;
@@ -266,7 +281,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
         pdl_wait();
         for (int j = 0; j < pre; ++j, ++it) {
           const uint32_t dst = smem_u32(smem + size_t(j) * kGuStageBytes);
-          tma_load_2d(dst + kGuWBytes, &tmA, full_bar(j), g * 128, 0);
+          tma_load_2d(dst + kGuWBytes, &tmA, full_bar(j), g * kX, 0);
           last_it[j] = it;
           if (++g == G) {
             g = 0;
@@ -281,8 +296,8 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
         if (!mbar_wait_bounded(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, &g_status)) break;
         const uint32_t dst = smem_u32(smem + size_t(s) * kGuStageBytes);
         mbar_arrive_expect_tx(full_bar(s), kTx);
-        tma_load_2d(dst, &tmW, full_bar(s), g * 128, b * kGuRows);
-        tma_load_2d(dst + kGuWBytes, &tmA, full_bar(s), g * 128, 0);
+        tma_load_2d(dst, &tmW, full_bar(s), g * kX, b * kGuRows);
+        tma_load_2d(dst + kGuWBytes, &tmA, full_bar(s), g * kX, 0);
         last_it[s] = it;
         if (++g == G) {
           g = 0;
@@ -321,7 +336,12 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
         const uint64_t bdesc = sw128_kmajor_desc(st + kGuWBytes);
         const uint32_t d_tmem = tmem_base + uint32_t(buf * kGuSlots);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_f8f6f4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kGuIdesc, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) {  // 32 bytes of K per MMA: 32 e4m3 or 16 bf16
+          if constexpr (kBf16)
+            umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kGuIdescBf16, kk > 0);
+          else
+            umma_f8f6f4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kGuIdesc, kk > 0);
+        }
         issued = true;
         umma_commit(empty_bar(s));    // the stage's bytes are consumed once these MMAs complete
         umma_commit(tfull_bar(buf));  // the unit's partial is in TMEM
@@ -346,7 +366,9 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
     // producer's weight prefetch, which waits on the ordering barrier) and a_scale as
     // [G][NT] (written by the previous kernel: after the grid-dependency wait), each
     // thread's loads issued together.
-    if (p.static_w) {
+    if (kBf16) {
+      pdl_wait();  // the activations and the workspace come from earlier kernels
+    } else if (p.static_w) {  // (fp8 only: the bf16 GEMM has no static-weight flag)
       float v[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) v[k] = et + 128 * k < n_units ? __ldg(p.w_scale + u0 + et + 128 * k) : 0.f;
@@ -361,7 +383,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
       for (int j = et; j < n_units; j += 128) sw_s[j] = __ldg(p.w_scale + u0 + j);
     }
     constexpr int kPer = 8;
-    for (int base = 0; base < NT * int(G); base += 128 * kPer) {
+    for (int base = 0; base < (kBf16 ? 0 : NT * int(G)); base += 128 * kPer) {
       float v[kPer];
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
@@ -393,6 +415,10 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(buf));  // the buffer may take the next unit
+      if constexpr (kBf16) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) acc[t] += __uint_as_float(d[t]);
+      } else {
       const float sw = sw_s[it];
       const float* sa = sa_s + g * NT;
 #pragma unroll
@@ -403,6 +429,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
         acc[t + 2] = fmaf(__uint_as_float(d[t + 2]), s4.z * sw, acc[t + 2]);
         acc[t + 3] = fmaf(__uint_as_float(d[t + 3]), s4.w * sw, acc[t + 3]);
       }
+      }
       if (g == G - 1 || it == n_units - 1) {
         // ---- block b ends here (or the CTA's range does)
         const bool whole = int64_t(b) * G >= u0 && g == G - 1;
@@ -411,7 +438,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
           if (n < p.N) {
 #pragma unroll
             for (int t = 0; t < NT; ++t)
-              if (t < p.M) p.out[int64_t(t) * p.N + n] = __float2bfloat16_rn(acc[t]);
+              if (t < p.M) gu_put(p, int64_t(t) * p.N + n, acc[t]);
           }
         } else {
           // partial sum: a plain store now, published after the loop
@@ -462,53 +489,60 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
 }
 
 // ---------------------------------------------------------------- host side
-static int gu_ctas(int64_t N, int64_t K) {
-  const int64_t units = ((N + kGuRows - 1) / kGuRows) * (K / 128);
-  return int(std::min<int64_t>(device_sm_count(), units));
+static int gu_ctas(int64_t N, int64_t K, bool bf16) {
+  const int64_t units = ((N + kGuRows - 1) / kGuRows) * (K / (bf16 ? 64 : 128));
+  return int(std::max<int64_t>(1, std::min<int64_t>(device_sm_count(), units / kGuMinUnitsPerCta)));
 }
 
 static bool gu_scales_fit(int64_t M, int64_t N, int64_t K) {
   const int64_t G = K / 128;
   const int64_t units = ((N + kGuRows - 1) / kGuRows) * G;
-  const int64_t ctas = gu_ctas(N, K);
+  const int64_t ctas = gu_ctas(N, K, false);
   const int64_t max_units = (units + ctas - 1) / ctas;
   const int64_t nt = M <= 8 ? 8 : M <= 16 ? 16 : 32;
   return (G * nt + max_units) * int64_t(sizeof(float)) <= kGuScaleBytes;
 }
 
-size_t gemv_umma_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  const size_t own = kCounterBytes + size_t(2) * gu_ctas(N, K) * kGuSlots * kGuRows * sizeof(float);
-  return std::max(own, gemv_tma_workspace_bytes(M, N, K));  // shapes whose scales do not fit take that kernel
+static size_t gu_own_workspace(int64_t N, int64_t K, bool bf16) {
+  return kCounterBytes + size_t(2) * gu_ctas(N, K, bf16) * kGuSlots * kGuRows * sizeof(float);
 }
 
-template <int NT>
+size_t gemv_umma_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  return std::max(gu_own_workspace(N, K, false), gemv_tma_workspace_bytes(M, N, K));  // fallback kernel's need
+}
+
+size_t gemv_umma_bf16_workspace_bytes(int64_t, int64_t N, int64_t K) { return gu_own_workspace(N, K, true); }
+
+template <int NT, bool kBf16>
 static int launch_gu(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out, int64_t M,
-                     int64_t N, int64_t K, void* ws, int static_w, void* stream) {
+                     int64_t N, int64_t K, void* ws, int static_w, int out_fp32, void* stream) {
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(gemv_umma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGuSmemBytes));
+    attr = cudaFuncSetAttribute(gemv_umma_kernel<NT, kBf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(kGuSmemBytes));
     if (attr == cudaSuccess)
-      attr = cudaFuncSetAttribute(gemv_umma_kernel<NT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+      attr = cudaFuncSetAttribute(gemv_umma_kernel<NT, kBf16>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                   int(cudaSharedmemCarveoutMaxShared));
   });
   if (attr != cudaSuccess) return int(attr);
   CUtensorMap mw, ma;
-  if (!make_tma_2d_kmajor(&mw, W, true, N, K, kGuRows) || !make_tma_2d_kmajor(&ma, A, true, M, K, NT))
+  if (!make_tma_2d_kmajor(&mw, W, !kBf16, N, K, kGuRows) || !make_tma_2d_kmajor(&ma, A, !kBf16, M, K, NT))
     return int(cudaErrorInvalidValue);
   GuParams p{};
   p.a_scale = a_scale;
   p.w_scale = w_scale;
-  p.out = static_cast<__nv_bfloat16*>(out);
+  p.out = out;
   p.M = int(M);
   p.N = int(N);
-  p.G = int(K / 128);
+  p.G = int(K / (kBf16 ? 64 : 128));
   p.nblk = int((N + kGuRows - 1) / kGuRows);
-  p.n_ctas = gu_ctas(N, K);
-  p.static_w = static_w;
+  p.n_ctas = gu_ctas(N, K, kBf16);
+  p.static_w = kBf16 ? 0 : static_w;
+  p.out_fp32 = kBf16 ? out_fp32 : 0;
   p.counter = static_cast<unsigned*>(ws);
   p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
-  return launch_kernel(gemv_umma_kernel<NT>, dim3(p.n_ctas), dim3(kGuThreads), kGuSmemBytes, stream, mw, ma, p);
+  return launch_kernel(gemv_umma_kernel<NT, kBf16>, dim3(p.n_ctas), dim3(kGuThreads), kGuSmemBytes, stream, mw, ma, p);
 }
 
 int launch_gemv_umma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
@@ -516,9 +550,18 @@ int launch_gemv_umma_a8w8(const void* A, const float* a_scale, const void* W, co
   if (M < 1 || M > kGemvMaxM || (N + kGuRows - 1) / kGuRows > kMaxCounters) return int(cudaErrorInvalidValue);
   if (!gu_scales_fit(M, N, K))
     return launch_gemv_tma_a8w8(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
-  if (M <= 8) return launch_gu<8>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
-  if (M <= 16) return launch_gu<16>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
-  return launch_gu<32>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
+  if (M <= 8) return launch_gu<8, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, 0, stream);
+  if (M <= 16) return launch_gu<16, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, 0, stream);
+  return launch_gu<32, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, 0, stream);
+}
+
+int launch_gemv_umma_bf16(const void* A, const void* W, void* out, int out_fp32, int64_t M, int64_t N, int64_t K,
+                          void* ws, void* stream) {
+  if (M < 1 || M > kGemvMaxM || K % 64 != 0 || (N + kGuRows - 1) / kGuRows > kMaxCounters)
+    return int(cudaErrorInvalidValue);
+  if (M <= 8) return launch_gu<8, true>(A, nullptr, W, nullptr, out, M, N, K, ws, 0, out_fp32, stream);
+  if (M <= 16) return launch_gu<16, true>(A, nullptr, W, nullptr, out, M, N, K, ws, 0, out_fp32, stream);
+  return launch_gu<32, true>(A, nullptr, W, nullptr, out, M, N, K, ws, 0, out_fp32, stream);
 }
 
 }  // namespace fp8bs

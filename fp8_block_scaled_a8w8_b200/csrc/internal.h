@@ -75,6 +75,9 @@ int launch_gemv_tma_a8w8(const void* A, const float* a_scale, const void* W, con
 size_t gemv_umma_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int launch_gemv_umma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
                           int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream);
+size_t gemv_umma_bf16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int launch_gemv_umma_bf16(const void* A, const void* W, void* out, int out_fp32, int64_t M, int64_t N, int64_t K,
+                          void* ws, void* stream);
 
 // Launch a kernel on a stream with programmatic stream serialisation (PDL) unless the
 // environment sets FP8BS_PDL=0. Returns the cudaError_t of the launch as int.

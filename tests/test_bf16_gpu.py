@@ -36,11 +36,24 @@ def test_bf16_parity(M, N, K, out_fp32):
 
 
 @pytest.mark.parametrize("cfg", ["bf16_tc_bn32", "bf16_tc_bn64", "bf16_tc_bn128", "bf16_tc_bn192", "bf16_tc_bn256",
-                                 "bf16_gemv_d2", "bf16_gemv_d4"])
+                                 "bf16_gemv_d2", "bf16_gemv_d4", "bf16_gemv_umma"])
 def test_bf16_configs(cfg):
     M = 20 if "gemv" in cfg else 200
     y, A, W = _run(M, 384, 640, False, seed=5, cfg=cfg)
     check_bf16(y, A, W, False)
+
+
+@pytest.mark.parametrize("M,N,K,out_fp32", [(1, 1024, 5120, True), (9, 144, 1344, False), (32, 4096, 64, True),
+                                            (5, 16, 6144, False)])
+def test_bf16_weight_streaming_tcgen05(M, N, K, out_fp32):
+    """The tcgen05 weight-streaming kernel: fp32 and bf16 out, N tails inside a 128-row block,
+    a single 64-column chunk, and a weight small enough that few CTAs share it; two calls
+    in a row give the same bits (fixed-order split-K sums)."""
+    y, A, W = _run(M, N, K, out_fp32, seed=M + 3, cfg="bf16_gemv_umma")
+    check_bf16(y, A, W, out_fp32)
+    y2, _, _ = _run(M, N, K, out_fp32, seed=M + 3, cfg="bf16_gemv_umma")
+    assert torch.equal(y.view(torch.int16) if not out_fp32 else y.view(torch.int32),
+                       y2.view(torch.int16) if not out_fp32 else y2.view(torch.int32))
 
 
 @pytest.mark.parametrize("M", [4096, 16384])
