@@ -76,6 +76,17 @@ def a8w8_bytes(M, N, K):
     return M * K + 4 * M * G + N * K + 4 * ((N + 127) // 128) * G + 2 * M * N
 
 
+def max_over_ranks(value_ms, device):
+    """The job's time is the slowest replica's: all-reduce MAX over the process group (any
+    backend; a no-op without one)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value_ms)], device=device, dtype=torch.float64)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def bf16_bytes(M, N, K, out_fp32):
     return 2 * M * K + 2 * N * K + (4 if out_fp32 else 2) * M * N
 
@@ -294,10 +305,7 @@ def run_gpu(args):
     quant_block_ms = float(np.mean([events[ph][2].elapsed_time(events[ph][0]) for ph in sorted(
         {(args.warmup + s) % period for s in range(args.steps)})]))
 
-    t = torch.tensor([step_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms = float(t.item())
+    step_ms = max_over_ranks(step_ms, dev)
 
     # ---- end to end through the public API: pinned host inputs in, results out, per step
     e2e = None
@@ -333,11 +341,7 @@ def run_gpu(args):
             e2e_step(s)
         e1.record(stream)
         barrier()
-        e2e_ms = e0.elapsed_time(e1) / e2e_steps
-        te = torch.tensor([e2e_ms], device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
         e2e = {"value": round(e2e_ms * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "api": "fp8_block_scaled_a8w8_b200.quant_act_per_token_group + gemm_a8w8_blockscale (eager)"}
@@ -623,11 +627,7 @@ def run_gpu_bf16(args):
     t_end.record(stream)
     barrier()
     clk = clocks.stop() if rank == 0 else None
-    step_ms = t_start.elapsed_time(t_end) / args.steps
-    t = torch.tensor([step_ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms = float(t.item())
+    step_ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, dev)
 
     e2e = None
     if args.e2e_steps > 0:
@@ -659,10 +659,8 @@ def run_gpu_bf16(args):
             e2e_step(s)
         e1.record(stream)
         barrier()
-        te = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": round(float(te.item()) * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+        e2e = {"value": round(e2e_ms * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "api": "fp8_block_scaled_a8w8_b200.gemm_bf16 (eager)"}
 
