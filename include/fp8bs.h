@@ -98,11 +98,12 @@ fp8bs_status fp8bs_quant_weight_block128(const float* w_f32, int64_t N, int64_t 
  * number of calls of any shapes issued in order on one stream. Calls that may run
  * concurrently need separate workspaces. After a call reported FP8BS_ERR_TIMEOUT
  * (fp8bs_get_device_status) the workspace must be zero-filled again.
- * The kernel is picked by the dispatch table (fp8bs_dispatch_lookup): a
- * weight-streaming split-K kernel for small M, a tcgen05/TMEM tensor-core kernel
- * fed by TMA otherwise. Results are deterministic (split-K partial sums are
- * reduced in a fixed order) and within the float32-accumulation bound of the
- * float64 oracle rounded once to bf16.
+ * The kernel is picked by the dispatch table (fp8bs_dispatch_lookup): for M <= 32 a
+ * weight-streaming split-K kernel (tcgen05 products, TMA-fed, stream-K over 128-row x
+ * 128-column units), otherwise a tiled tcgen05/TMEM kernel fed by TMA, which also splits
+ * K when its output tiles would leave most SMs idle (then it needs workspace too).
+ * Results are deterministic (split-K partial sums are reduced in a fixed order) and
+ * within the float32-accumulation bound of the float64 oracle rounded once to bf16.
  */
 fp8bs_status fp8bs_gemm_a8w8_blockscale(const void* A_e4m3, const float* a_scale, const void* W_e4m3,
                                         const float* w_scale, void* out_bf16, int64_t M, int64_t N,
