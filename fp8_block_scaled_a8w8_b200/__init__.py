@@ -153,9 +153,14 @@ def workspace_bytes(op: int, M: int, N: int, K: int) -> int:
 
 
 class Workspace:
-    """A zero-filled device scratch buffer that grows on demand (torch allocates it; the
-    library only uses it). The library leaves it zero-filled after every call, so one
-    instance serves any number of calls issued on one stream."""
+    """A device scratch buffer, zero-filled when allocated, that grows on demand (torch
+    allocates it; the library only uses it). Every call leaves its split-K arrival counters
+    at zero and overwrites partial sums before reading them, so one instance serves any
+    number of calls issued in order on one stream.
+
+    Growing replaces the buffer: the device is synchronised before (no kernel still uses the
+    old one) and after the zero fill (every stream sees the zeros). Growing is refused
+    during CUDA-graph capture: size the workspace with an eager call first, or pass one."""
 
     def __init__(self, device=None):
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
@@ -165,7 +170,12 @@ class Workspace:
         if nbytes == 0:
             return None
         if self.buf is None or self.buf.numel() < nbytes:
+            if torch.cuda.is_current_stream_capturing():
+                raise RuntimeError("the default workspace cannot grow during CUDA-graph capture: make one eager "
+                                   "call of this shape first, or pass workspace=")
+            torch.cuda.synchronize(self.device)
             self.buf = torch.zeros(((nbytes + 255) // 256) * 256, dtype=torch.uint8, device=self.device)
+            torch.cuda.synchronize(self.device)
         return self.buf
 
 
