@@ -34,6 +34,9 @@
  *    calls return FP8BS_ERR_CUDA or FP8BS_ERR_UNSUPPORTED.
  *  - No C++ exception crosses this interface. All functions are thread-safe;
  *    the dispatch table's counters are process-global atomics.
+ *  - One device per process (one process per GPU): kernel attributes such as the
+ *    dynamic shared-memory size are set once, in the context of the device that is
+ *    current at a kernel's first launch.
  */
 #ifndef FP8BS_H
 #define FP8BS_H
