@@ -41,6 +41,34 @@ def _headers():
 # would wait for registers that do not exist), so the build checks it.
 REGISTER_CONTRACTS = {"gemm_tc.cu": ("gemm_tc_kernel", 168)}
 
+# Hot kernels that must compile without register spills (mangled-name patterns): the
+# decode kernels, the one-split tensor-core kernel and the mma.sync decode kernel with
+# staged scales. The split-K tensor-core instantiations and rare fallbacks may spill a few
+# bytes and are not listed.
+SPILL_FREE = {"gemv_umma.cu": [r"gemv_umma_kernel"], "gemm_tc.cu": [r"gemm_tc_kernel.*Lb0EEEv"],
+              "gemv_tma.cu": [r"gemv_tma_kernel.*Lb1EEEv"]}
+
+
+def _check_spill_free(src: str, log: str) -> None:
+    pats = [re.compile(p) for p in SPILL_FREE.get(src, [])]
+    if not pats:
+        return
+    lines = log.splitlines()
+    seen = 0
+    for i, line in enumerate(lines):
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if not m or not any(p.search(m.group(1)) for p in pats):
+            continue
+        for nxt in lines[i + 1:i + 6]:
+            sm = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", nxt)
+            if sm:
+                seen += 1
+                if int(sm.group(1)) or int(sm.group(2)):
+                    raise RuntimeError(f"{src}: {m.group(1)} spills ({nxt.strip()})")
+                break
+    if seen == 0:
+        raise RuntimeError(f"{src}: no ptxas spill report for {SPILL_FREE[src]}")
+
 
 def _check_register_contract(src: str, log: str) -> None:
     if src not in REGISTER_CONTRACTS:
@@ -71,13 +99,14 @@ def _compile(src: str, force: bool, ptxas_verbose: bool) -> tuple[str, str]:
     cmd = [NVCC, *ARCH, *COMMON, "-c", path, "-o", obj]
     if src.endswith(".cpp"):
         cmd[1:1] = ["-x", "cu"]
-    if (ptxas_verbose and src.endswith(".cu")) or src in REGISTER_CONTRACTS:
+    if (ptxas_verbose and src.endswith(".cu")) or src in REGISTER_CONTRACTS or src in SPILL_FREE:
         cmd.append("-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
     try:
         _check_register_contract(src, r.stderr)
+        _check_spill_free(src, r.stderr)
     except RuntimeError:
         os.remove(obj)
         raise
