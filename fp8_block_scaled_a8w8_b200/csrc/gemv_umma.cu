@@ -22,7 +22,7 @@
 // groups). The tensor core runs up to eight units ahead of the epilogue.
 //
 //   warp 0        TMA producer: per unit one weight box (128 rows x 128 bytes) and one
-//                 token box (32 rows x 128 bytes); with static weights the first few
+//                 token box (NT rows x 128 bytes); with static weights the first few
 //                 weight boxes are fetched before the grid-dependency wait
 //   warp 1        TMEM allocator; lane 0 issues the MMAs of even units
 //   warp 2        lane 0 issues the MMAs of odd units
@@ -33,6 +33,15 @@
 // columns, zero past M; its run of w_scale, which is [nblk, G] row-major, so unit u's
 // weight scale is w_scale[u]); shapes whose scales do not fit the staging region go to
 // the mma.sync kernel instead.
+//
+// A CTA uses 112 KB of shared memory and 256 TMEM columns, so two fit on an SM: the
+// next call's CTAs become resident while this call's still stream and fetch their first
+// weight boxes during its tail. Every CTA takes at least 8 units (small weights are not
+// split into dozens of contributors per block).
+//
+// The bf16 GEMM (kBf16) runs the same kernel: a unit is 128 weight rows x 64 bf16
+// columns (the same 128-byte rows), the products are kind::f16, there are no scales, and
+// the output may be float32.
 //
 // Every wait is bounded (kWaitLimitNs); on expiry the CTA raises its abort flag and the
 // device status word, every role leaves its loop, in-flight TMA copies and MMAs are
