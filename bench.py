@@ -18,7 +18,7 @@ timed region is bracketed by a barrier and a device synchronise on both sides an
 the step time is the max over ranks. N>1 runs N independent replicas (the path
 has no exchange step).
 
---impl reference times the CPU oracle (the only other arm this build has) on a
+--impl reference times the CPU oracle (the only other arm there is) on a
 bounded sample of the same workload, on the host cores.
 """
 

@@ -77,7 +77,7 @@ def weight_bf16(N: int, K: int, seed: int, sigma: float = SIGMA_W) -> torch.Tens
     return weight_f32(N, K, seed, sigma).to(torch.bfloat16)
 
 
-def config0(seed: int = 0):
+def m1_n5120_k6144(seed: int = 0):
     """Single GEMM M=1, N=5120, K=6144: one generator, A drawn first, then W."""
     M, N, K = 1, 5120, 6144
     rng = np.random.default_rng(seed)

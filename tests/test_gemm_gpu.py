@@ -135,10 +135,10 @@ def test_deterministic_and_graph_replay(M, N, K):
     check_a8w8(y1, *case)
 
 
-def test_config0_end_to_end():
+def test_m1_n5120_k6144_end_to_end():
     """M=1, N=5120, K=6144, seed 0: bf16 activations and float32 weights quantised on the
     GPU, then the GEMM; the oracle quantises and multiplies on its own."""
-    x, w = inputs.config0(0)
+    x, w = inputs.m1_n5120_k6144(0)
     q, s = fb.quant_act_per_token_group(x.cuda())
     wq, ws = fb.quant_weight_block128(w.cuda())
     y = fb.gemm_a8w8_blockscale(q, s, wq, ws)

@@ -130,7 +130,7 @@ def test_bf16_rounding_floor_matches_pages(golden_dir):
     floor = dict(l.split() for l in open(os.path.join(golden_dir, "accuracy_floor.txt"))
                  if l.strip() and not l.startswith("#"))
     page = float(floor["bf16_output_rounding_floor"])
-    x, w = inputs.config0(0)
+    x, w = inputs.m1_n5120_k6144(0)
     A_q, a_s = quant.quant_act_per_token_group(x.float().numpy())
     W_q, w_s = quant.quant_weight_block128(w.numpy())
     ref, out = gemm.gemm_a8w8_blockscale(A_q, a_s, W_q, w_s)
