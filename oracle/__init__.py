@@ -34,7 +34,7 @@ Modules:
   bf16      -- round-to-nearest-even to bfloat16 from float64
   quant     -- per-token 1x128 activation quantiser, 128x128 weight quantiser
   gemm      -- a8w8 block-scaled GEMM and plain bf16 GEMM in float64
-  metrics   -- relative L2, error ratio, element-wise bound
+  metrics   -- relative L2, error ratio, bf16 ulp
   dispatch  -- the padded-M lookup walk and the census deduplication rule
 
 Parity status of every function is listed in each module's header; every
