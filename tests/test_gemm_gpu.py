@@ -165,22 +165,97 @@ def test_decode_sweep_full_size(nk_index):
         check_a8w8(y, A_q, a_s, W_q, w_s)
 
 
-@pytest.mark.parametrize("M", [2048, 6016, 8192])
-def test_prefill_full_size_sampled_rows(M):
-    N, K = inputs.PREFILL_NK[1]  # (34816, 5120)
-    w = inputs.weight_f32(N, K, 11)
-    x = inputs.activation_bf16(M, K, 12 + M, outliers=True)
-    wq, ws = fb.quant_weight_block128(w.cuda())
+_PREFILL_W = {}
+
+
+def _prefill_weight(nk_index):
+    """Quantised prefill weight: GPU codes and scales, and the oracle's own quantisation."""
+    if nk_index not in _PREFILL_W:
+        _PREFILL_W.clear()  # one (N, K) at a time: 34816 x 5120 in float64 is 1.4 GB
+        N, K = inputs.PREFILL_NK[nk_index]
+        w = inputs.weight_f32(N, K, 11 + nk_index)
+        wq, ws = fb.quant_weight_block128(w.cuda())
+        W_q, w_s = oquant.quant_weight_block128(w.numpy())
+        _PREFILL_W[nk_index] = (wq, ws, W_q, w_s)
+    return _PREFILL_W[nk_index]
+
+
+def prefill_rows(M, seed, count=256):
+    """The first and last rows, every row of the last 128-row tile (the M tail when
+    M % 128 != 0), the rows on both sides of a few tile boundaries, and seeded random rows
+    up to `count`."""
+    rng = np.random.default_rng(seed)
+    last_tile = ((M - 1) // 128) * 128
+    fixed = set(range(0, 8)) | set(range(last_tile, M)) | {M - 1}
+    for t in rng.choice(max(1, M // 128), min(8, max(1, M // 128)), replace=False):
+        fixed |= {int(t) * 128 - 1, int(t) * 128} if t > 0 else {0}
+    fixed = {r for r in fixed if 0 <= r < M}
+    rest = np.setdiff1d(np.arange(M), np.fromiter(fixed, dtype=np.int64))
+    extra = rng.choice(rest, max(0, min(count - len(fixed), rest.size)), replace=False) if rest.size else []
+    return np.unique(np.concatenate([np.fromiter(fixed, dtype=np.int64), np.asarray(extra, dtype=np.int64)]))
+
+
+@pytest.mark.parametrize("M", inputs.PREFILL_MS)
+@pytest.mark.parametrize("nk_index", [0, 1])
+def test_prefill_full_size_sampled_rows(M, nk_index):
+    """Prefill shapes at full size (1% outlier channels x20), checked on 256 rows against the
+    oracle: first and last rows, the last 128-row tile, tile-boundary rows, random rows."""
+    N, K = inputs.PREFILL_NK[nk_index]
+    wq, ws, W_q, w_s = _prefill_weight(nk_index)
+    x = inputs.activation_bf16(M, K, 12 + M + nk_index, outliers=True)
     q, s = fb.quant_act_per_token_group(x.cuda())
     y = fb.gemm_a8w8_blockscale(q, s, wq, ws)
     torch.cuda.synchronize()
-    rng = np.random.default_rng(M)
-    rows = np.unique(np.concatenate([[0, 1, 127, 128, M - 1, M - 2, (M // 128) * 128 - 1],
-                                     rng.choice(M, 9, replace=False)]))
-    rows = rows[rows < M]
-    W_q, w_s = oquant.quant_weight_block128(w.numpy())
+    assert fb.get_device_status() == 0
+    rows = prefill_rows(M, seed=M + nk_index)
+    assert rows.size == 256
     A_q, a_s = oquant.quant_act_per_token_group(x.float().numpy()[rows])
+    assert np.array_equal(codes_from_device(q)[rows], A_q)
     check_a8w8(y.cpu()[torch.from_numpy(rows)], A_q, a_s, W_q, w_s)
+
+
+def test_prefill_m2048_n14336_full_matrix():
+    """Every output of the M = 2048, N = 14336, K = 5120 prefill call against the oracle
+    (checked 256 rows at a time)."""
+    M = 2048
+    N, K = inputs.PREFILL_NK[0]
+    wq, ws, W_q, w_s = _prefill_weight(0)
+    x = inputs.activation_bf16(M, K, 12 + M, outliers=True)
+    q, s = fb.quant_act_per_token_group(x.cuda())
+    y = fb.gemm_a8w8_blockscale(q, s, wq, ws)
+    torch.cuda.synchronize()
+    assert fb.get_device_status() == 0
+    A_q, a_s = oquant.quant_act_per_token_group(x.float().numpy())
+    yc = y.cpu()
+    for r0 in range(0, M, 256):
+        check_a8w8(yc[r0:r0 + 256], A_q[r0:r0 + 256], a_s[r0:r0 + 256], W_q, w_s)
+
+
+def test_ladder_every_tile_tail_class():
+    """The dense-M ladder on (5120, 6144): one M from every residue class mod 128 in
+    257..8192 (seeded), each checked on its last 128-row tile -- the M-tail rows -- and
+    its first rows. The activations of all calls are row prefixes of one quantised
+    8192 x 6144 matrix."""
+    N, K = inputs.LADDER_NK
+    w = inputs.weight_f32(N, K, 31)
+    wq, ws = fb.quant_weight_block128(w.cuda())
+    W_q, w_s = oquant.quant_weight_block128(w.numpy())
+    x = inputs.activation_bf16(8192, K, 32)
+    q, s = fb.quant_act_per_token_group(x.cuda())
+    rng = np.random.default_rng(33)
+    ms = sorted(257 + r + 128 * int(rng.integers(0, (8192 - 257 - r) // 128 + 1)) for r in range(128))
+    assert len({m % 128 for m in ms}) == 128 and max(ms) <= 8192
+    rows_of = {M: np.concatenate([np.arange(0, 2), np.arange(((M - 1) // 128) * 128, M)]) for M in ms}
+    ys = {}
+    for M in ms:
+        y = fb.gemm_a8w8_blockscale(q[:M], s[:M], wq, ws)
+        ys[M] = y[torch.from_numpy(rows_of[M]).cuda()].cpu()
+    torch.cuda.synchronize()
+    assert fb.get_device_status() == 0
+    xf = x.float().numpy()
+    for M in ms:
+        A_q, a_s = oquant.quant_act_per_token_group(xf[rows_of[M]])
+        check_a8w8(ys[M], A_q, a_s, W_q, w_s)
 
 
 def test_workspace_shared_across_shapes():
