@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-Default workload (N=1): the decode sweep -- M in {1,2,3,4,8,9,16} on the four
+Headline workload (N=1): the decode sweep -- M in {1,2,3,4,8,9,16} on the four
 Qwen3.8-27B projections (N,K) = (5120,6144), (14336,5120), (16384,5120),
 (34816,5120) of [aiter#7752] "Kernel". One step is one pass of the hot path over
 the sweep: for each of the 28 (M,N,K) calls, per-token 1x128 activation
@@ -17,6 +17,13 @@ replayed; CUDA events recorded inside the graphs time every GEMM launch. The
 timed region is bracketed by a barrier and a device synchronise on both sides and
 the step time is the max over ranks. N>1 runs N independent replicas (the path
 has no exchange step).
+
+The default run also measures, with a few steps each, every other configuration: the
+prefill shapes, the dense M ladder (with the dispatch census and its padded-M drift) and
+the bf16 small-N GEMMs, each as an entry of "workloads" with its own roofline; the
+per-shape "detail" table gives cold- and hot-weight us/call, and the CPU leg reports the
+oracle's time and the accuracy of the timed outputs against it. --only skips the extra
+workloads.
 
 --impl reference times the CPU oracle (the only other arm there is) on a
 bounded sample of the same workload, on the host cores.
@@ -166,11 +173,10 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- GPU arm
-def run_gpu(args):
+def init_gpu():
+    """One process per GPU: (world, rank, device); NCCL process group for N > 1."""
     import torch
     import torch.distributed as dist
-
-    import fp8_block_scaled_a8w8_b200 as fb
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -181,11 +187,20 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
-    dev = torch.device("cuda", torch.cuda.current_device())
+    return world, rank, torch.device("cuda", torch.cuda.current_device())
+
+
+def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail, e2e_steps, cpu):
+    """The JSON line of one a8w8 workload (rank 0; None elsewhere). Every rank takes the
+    same collective steps."""
+    import torch
+    import torch.distributed as dist
+
+    import fp8_block_scaled_a8w8_b200 as fb
+
     fb.lib()
     pk = peaks()
-
-    calls = workload_calls(args.workload, args.shape)
+    calls = workload_calls(workload, shape)
     uses = {}
     for (M, N, K, i, j, o) in calls:
         uses[(N, K)] = uses.get((N, K), 0) + 1
@@ -279,7 +294,7 @@ def run_gpu(args):
         torch.cuda.synchronize()
 
     with torch.cuda.stream(stream):
-        for s in range(args.warmup):
+        for s in range(warmup):
             graphs[s % period].replay()
     barrier()
 
@@ -290,26 +305,26 @@ def run_gpu(args):
     t_end = torch.cuda.Event(enable_timing=True)
     barrier()
     t_start.record(stream)
-    for s in range(args.steps):
+    for s in range(steps):
         with torch.cuda.stream(stream):
-            graphs[(args.warmup + s) % period].replay()
+            graphs[(warmup + s) % period].replay()
     t_end.record(stream)
     barrier()
     clk = clocks.stop() if rank == 0 else None
-    step_ms = t_start.elapsed_time(t_end) / args.steps
+    step_ms = t_start.elapsed_time(t_end) / steps
 
     # average GEMM launch duration: the GEMM block of the last replay of every phase
     gemm_block_ms = [events[ph][0].elapsed_time(events[ph][1]) for ph in sorted(
-        {(args.warmup + s) % period for s in range(args.steps)})]
+        {(warmup + s) % period for s in range(steps)})]
     gemm_ms_per_call = float(np.mean(gemm_block_ms)) / n_calls
     quant_block_ms = float(np.mean([events[ph][2].elapsed_time(events[ph][0]) for ph in sorted(
-        {(args.warmup + s) % period for s in range(args.steps)})]))
+        {(warmup + s) % period for s in range(steps)})]))
 
     step_ms = max_over_ranks(step_ms, dev)
 
     # ---- end to end through the public API: pinned host inputs in, results out, per step
     e2e = None
-    e2e_steps = args.e2e_steps if n_calls <= 64 and max(maxm.values()) <= 64 else min(args.e2e_steps, 3)
+    e2e_steps = e2e_steps if n_calls <= 64 and max(maxm.values()) <= 64 else min(e2e_steps, 3)
     if e2e_steps > 0:
         hx = [x.cpu().pin_memory() for x in xs]
         hy = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
@@ -347,8 +362,8 @@ def run_gpu(args):
                "api": "fp8_block_scaled_a8w8_b200.quant_act_per_token_group + gemm_a8w8_blockscale (eager)"}
 
     if rank == 0:
-        detail = per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk) \
-            if args.detail else None
+        det = per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk) \
+            if detail else None
         tot_bytes = float(sum(a8w8_bytes(M, N, K) for (M, N, K, *_r) in calls))
         tot_ms = gemm_ms_per_call * n_calls
         tot_flops = sum(2.0 * M * N * K for (M, N, K, *_r) in calls)
@@ -380,91 +395,139 @@ def run_gpu(args):
                       "us_per_step": round(quant_block_ms * 1000.0, 2),
                       "algorithmic_bytes_per_step": int(q_bytes),
                       "note": "bf16 read + e4m3 write + fp32 scales per element; at decode M the launches are latency-bound"}
-        cpu = cpu_baseline(args.workload) if (args.cpu_baseline and world == 1) else None
+        cpu_line = None
+        if cpu and world == 1:
+            def gpu_output(c, rows):
+                """The call's output recomputed through the public API on copy 0 of its weight
+                (the inputs of the timed calls), rows selected, as float64."""
+                M, N, K, *_r = calls[c]
+                wq0, ws0 = wcopies[(N, K)][0]
+                with torch.cuda.stream(stream):
+                    q, sc = fb.quant_act_per_token_group(xs[c], stream=stream)
+                    y = fb.gemm_a8w8_blockscale(q, sc, wq0, ws0, workspace=workspace, stream=stream)
+                stream.synchronize()
+                return y.float().cpu().numpy().astype(np.float64)[rows]
+            cpu_line = cpu_baseline(workload, calls, [x.cpu() for x in xs], gpu_output)
         line = {
             "metric": METRIC, "value": round(step_ms * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(step_ms, 4),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 -> bf16",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no dataset)",
-            "config": {"workload": args.workload if not args.shape else "shape " + args.shape,
-                       "description": inputs.WORKLOADS[args.workload] if not args.shape else "one a8w8 call shape M,N,K",
+            "config": {"workload": workload if not shape else "shape " + shape,
+                       "description": inputs.WORKLOADS[workload] if not shape else "one a8w8 call shape M,N,K",
                        "calls_per_step": n_calls,
                        "weight_rotation_mib": ROTATE_BYTES >> 20,
                        "l2": "working set per step >> 126 MB L2 (rotated weights); no flush needed",
                        "parallelism": f"replicas x{world}", "timing": "CUDA graphs replayed, CUDA events, max over ranks"},
             "roofline": roof, "quant_roofline": quant_roof,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * n_calls * args.steps,
-            "clocks": clk, "dispatch": {**census, "table_hash": fb.dispatch_table_hash()},
-            "detail": detail,
+            "cpu_baseline": cpu_line, "e2e": e2e, "gpu_launches": 2 * n_calls * steps,
+            "clocks": clk, "dispatch": {**census, "table_hash": fb.dispatch_table_hash(),
+                                        "padded_m_drift": padded_m_drift(fb.dispatch_dump_json(), fb.OP_A8W8_BLOCKSCALE)},
+            "detail": det,
         }
-        print(json.dumps(line), flush=True)
+        if cpu_line is not None and "accuracy" in cpu_line:
+            line["accuracy"] = cpu_line.pop("accuracy")
+        if det:
+            hot = [d["hot_us"] for d in det if d.get("hot_us") is not None]
+            per_shape = {(d["M"], d["N"], d["K"]): d for d in det}
+            cold_mean = float(np.mean([per_shape[(M, N, K)]["us"] for (M, N, K, *_r) in calls]))
+            hot_mean = float(np.mean([per_shape[(M, N, K)]["hot_us"] for (M, N, K, *_r) in calls])) if hot else None
+            line["hot"] = {"value": round(hot_mean, 3) if hot_mean else None, "unit": "µs/call",
+                           "cold_value": round(cold_mean, 3),
+                           "protocol": "GEMM only, 20 back-to-back calls per shape in a CUDA graph: hot = one weight "
+                                       "copy (L2-resident when it fits), cold = rotated over >= 512 MiB; mean over "
+                                       "the workload's calls"}
+            one = per_shape.get((1, 5120, 6144))
+            if one is not None:
+                line["single_call"] = {"workload": "decode_m1_n5120_k6144", "M": 1, "N": 5120, "K": 6144,
+                                       "us": one["us"], "hot_us": one.get("hot_us"), "GBps": one["GBps"],
+                                       "roofline_frac": one["roofline_frac"], "cfg": one["cfg"]}
+    else:
+        line = None
     for g in graphs:
         del g
     graphs.clear()
-    if world > 1:
-        dist.destroy_process_group()
+    return line
 
 
 def per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk, R=20, rounds=7):
-    """us/call of every distinct call shape: R back-to-back calls on rotated weight copies
-    in one CUDA graph, median over rounds interleaved across shapes ([aiter#7752] "Kernel":
-    graph replay, median of interleaved rounds)."""
+    """us/call of every distinct call shape: R back-to-back calls in one CUDA graph, median
+    over rounds interleaved across shapes ([aiter#7752] "Kernel": graph replay, median of
+    interleaved rounds), once on weight copies rotated over >= 512 MiB (cold: every call
+    reads its weights from HBM) and once on a single copy (hot), as the pages report both."""
     seen, idx = set(), []
     for c, (M, N, K, *_r) in enumerate(calls):
         if (M, N, K) not in seen:
             seen.add((M, N, K))
             idx.append(c)
-    graphs = []
+    graphs = {}
     with torch.cuda.stream(stream):
         for c in idx:
             M, N, K, *_r = calls[c]
             cp = wcopies[(N, K)]
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for r in range(R):
-                    wq, wsc = cp[r % len(cp)]
-                    fb.gemm_a8w8_blockscale(qs[c], ss[c], wq, wsc, out=outs[c], workspace=workspace, stream=stream,
-                                            static_weights=True)
-            graphs.append(g)
-    times = {c: [] for c in idx}
+            for kind in ("cold", "hot"):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for r in range(R):
+                        wq, wsc = cp[r % len(cp)] if kind == "cold" else cp[0]
+                        fb.gemm_a8w8_blockscale(qs[c], ss[c], wq, wsc, out=outs[c], workspace=workspace,
+                                                stream=stream, static_weights=True)
+                graphs[(c, kind)] = g
+    times = {k: [] for k in graphs}
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(rounds):
-        for c, g in zip(idx, graphs):
+        for k, g in graphs.items():
             with torch.cuda.stream(stream):
                 e0.record(stream)
                 g.replay()
                 e1.record(stream)
             e1.synchronize()
-            times[c].append(e0.elapsed_time(e1) * 1000.0 / R)
+            times[k].append(e0.elapsed_time(e1) * 1000.0 / R)
     out = []
     for c in idx:
         M, N, K, *_r = calls[c]
-        t = sorted(times[c])
+        t = sorted(times[(c, "cold")])
         us = t[len(t) // 2]
+        th = sorted(times[(c, "hot")])
         by = a8w8_bytes(M, N, K)
         fl = 2.0 * M * N * K
+        # timed alone in short bursts: the burst peaks (HBM copy; fp8 = 2 x burst bf16)
         roof_us = max(by / (pk["hbm_gbs"] * 1e3), fl / (2 * pk["bf16_tflops"] * 1e6))
         out.append({"M": M, "N": N, "K": K, "cfg": cfgs[c], "us": round(us, 3),
-                    "iqr_us": round(t[(3 * len(t)) // 4] - t[len(t) // 4], 3),
+                    "iqr_us": round(t[(3 * len(t)) // 4] - t[len(t) // 4], 3), "hot_us": round(th[len(th) // 2], 3),
                     "GBps": round(by / us / 1e3, 1), "TFLOPS": round(fl / us / 1e6, 2),
                     "roofline_frac": round(roof_us / us, 3)})
-    del graphs
+    graphs.clear()
     return out
 
 
+def padded_m_drift(census, op):
+    """Padded-M drift of the census ([cookbook#8] "Two amplifiers": M = 6016 runs the row
+    tuned for 8192): lookups whose hit came from a row at a padded M other than the exact
+    M, their share of all hits, and the distinct (M, padded_M) pairs."""
+    hits = [r for r in census if r["op"] == op and r["hit"]]
+    drifted = [r for r in hits if r["padded_M"] != r["M"]]
+    n_hits = sum(r["count"] for r in hits)
+    n_drift = sum(r["count"] for r in drifted)
+    return {"lookups": n_drift, "share_of_hits": round(n_drift / n_hits, 4) if n_hits else 0.0,
+            "distinct": len({(r["M"], r["padded_M"]) for r in drifted}),
+            "max_ratio": round(max((r["padded_M"] / r["M"] for r in drifted), default=1.0), 3)}
+
+
 # --------------------------------------------------------------------------- CPU oracle
-def _oracle_call(M, N, K, i, j, o, wcache):
+def _oracle_call(x, N, K, i, wcache):
+    """The oracle on one call: activations x (float32 array of bf16 values), the call's
+    weight quantised by the oracle (set-up, untimed). Returns (seconds, ref float64)."""
     from oracle import gemm as ogemm, quant as oquant
     key = (N, K)
     if key not in wcache:
         w = inputs.weight_f32(N, K, inputs.decode_seed_w(i)).numpy()
         wcache[key] = oquant.quant_weight_block128(w)  # set-up, untimed
-    x = inputs.activation_bf16(M, K, inputs.decode_seed_a(i, j), outliers=o).float().numpy()
     W_q, w_s = wcache[key]
     t0 = time.perf_counter()
     A_q, a_s = oquant.quant_act_per_token_group(x)
-    ogemm.gemm_a8w8_blockscale(A_q, a_s, W_q, w_s)
-    return time.perf_counter() - t0
+    ref, _ = ogemm.gemm_a8w8_blockscale(A_q, a_s, W_q, w_s)
+    return time.perf_counter() - t0, ref
 
 
 def _threads():
@@ -476,28 +539,68 @@ def _threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(workload, budget_s=20.0):
-    """The oracle as it stands, timed on the host on a bounded sample of the workload."""
-    calls = workload_calls(workload)
-    rng = np.random.default_rng(0)
-    order = list(rng.permutation(len(calls)))
+def _host():
+    """CPU model and the cores this process may run on (sched_getaffinity)."""
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    try:
+        aff = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        aff = os.cpu_count()
+    return {"cpu_model": model, "affinity_cores": aff}
+
+
+def _accuracy(pairs):
+    """rel L2 ([aiter#7752] "Kernel") and error ratio ([aiter#7247] "Test Result"; atol =
+    1e-2 x rms of the reference, rtol = 1e-2) of GPU outputs against the oracle, over all
+    compared outputs."""
+    from oracle import metrics as ometrics
+    y = np.concatenate([p[0].ravel() for p in pairs])
+    r = np.concatenate([p[1].ravel() for p in pairs])
+    rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
+    return {"rel_l2": round(ometrics.rel_l2(y, r), 6),
+            "error_ratio": round(ometrics.error_ratio(y, r, atol=1e-2 * rms, rtol=1e-2), 6),
+            "atol": round(1e-2 * rms, 8), "rtol": 1e-2, "outputs": int(y.size),
+            "reference": "CPU oracle in float64 (unrounded)"}
+
+
+def cpu_baseline(workload, calls=None, xs=None, gpu_output=None, budget_s=20.0):
+    """The oracle as it stands, timed on the host on a bounded sample of the workload. With
+    the timed calls' activations (xs) and a way to recompute a call's GPU output, the same
+    oracle results also give the accuracy of the GPU outputs on that sample."""
+    if calls is None:
+        calls = workload_calls(workload)
+    order = list(np.random.default_rng(0).permutation(len(calls)))
     wcache = {}
-    spent, n, done = 0.0, 0, []
+    spent, done, pairs = 0.0, [], []
     for c in order:
         M, N, K, i, j, o = calls[c]
-        if workload in ("prefill", "ladder") and M > 64:
-            M = 64  # rows of a large-M call: the oracle is row-separable; time per row is scaled below
-        dt = _oracle_call(M, N, K, i, j, o, wcache)
-        scale = calls[c][0] / M
+        m = min(M, 64)  # rows of a large-M call: the oracle is row-separable; time per row is scaled below
+        rows = np.arange(m) if m == M else np.unique(np.concatenate([np.arange(m // 2), np.arange(M - m + m // 2, M)]))
+        if xs is not None:
+            x = xs[c].float().numpy()[rows]
+        else:
+            x = inputs.activation_bf16(M, K, inputs.decode_seed_a(i, j), outliers=o).float().numpy()[rows]
+        dt, ref = _oracle_call(x, N, K, i, wcache)
+        if gpu_output is not None:
+            pairs.append((gpu_output(c, rows), ref))
         spent += dt
-        done.append(dt * scale)
-        n += 1
+        done.append(dt * M / len(rows))
         if spent > budget_s:
             break
     us = float(np.mean(done)) * 1e6
-    return {"value": round(us, 1), "unit": "µs/call", "cores": _threads(), "kind": "oracle",
-            "sample": f"{n} of {len(calls)} calls of the {workload} workload (random order), quant + GEMM in float64"
-                      f"{'; large-M calls timed on 64 rows and scaled by M/64' if workload in ('prefill', 'ladder') else ''}"}
+    out = {"value": round(us, 1), "unit": "µs/call", "cores": _threads(), **_host(), "kind": "oracle",
+           "sample": f"{len(done)} of {len(calls)} calls of the {workload} workload (random order), quant + GEMM in "
+                     f"float64{'; calls with M > 64 timed on 64 rows (first and last) and scaled by M/64' if any(c[0] > 64 for c in calls) else ''}"}
+    if pairs:
+        out["accuracy"] = {**_accuracy(pairs), "sample": f"the same {len(pairs)} calls, outputs of the timed inputs"}
+    return out
 
 
 # --------------------------------------------------------------------------- bf16 small-N workload
@@ -531,27 +634,19 @@ def cpu_baseline_bf16(budget_s=20.0):
         done.append(dt * M / m)
         if spent > budget_s:
             break
-    return {"value": round(float(np.mean(done)) * 1e6, 1), "unit": "µs/call", "cores": _threads(), "kind": "oracle",
+    return {"value": round(float(np.mean(done)) * 1e6, 1), "unit": "µs/call", "cores": _threads(), **_host(),
+            "kind": "oracle",
             "sample": f"{len(done)} of {len(calls)} calls of the bf16_small_n workload (random order), float64 "
                       "matmul; calls with M > 64 timed on 64 rows and scaled by M/64"}
 
 
-def run_gpu_bf16(args):
+def measure_bf16(args, world, rank, dev, steps, warmup, detail, e2e_steps, cpu):
+    """The JSON line of the bf16 small-N workload (rank 0; None elsewhere)."""
     import torch
     import torch.distributed as dist
 
     import fp8_block_scaled_a8w8_b200 as fb
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    dev = torch.device("cuda", torch.cuda.current_device())
     fb.lib()
     pk = peaks()
     calls = bf16_calls()
@@ -612,7 +707,7 @@ def run_gpu_bf16(args):
         torch.cuda.synchronize()
 
     with torch.cuda.stream(stream):
-        for s in range(args.warmup):
+        for s in range(warmup):
             graphs[s % period].replay()
     barrier()
     clocks = ClockSampler(dev.index)
@@ -621,17 +716,17 @@ def run_gpu_bf16(args):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     t_start.record(stream)
-    for s in range(args.steps):
+    for s in range(steps):
         with torch.cuda.stream(stream):
-            graphs[(args.warmup + s) % period].replay()
+            graphs[(warmup + s) % period].replay()
     t_end.record(stream)
     barrier()
     clk = clocks.stop() if rank == 0 else None
-    step_ms = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, dev)
+    step_ms = max_over_ranks(t_start.elapsed_time(t_end) / steps, dev)
 
     e2e = None
-    if args.e2e_steps > 0:
-        e2e_steps = min(args.e2e_steps, 5)
+    if e2e_steps > 0:
+        e2e_steps = min(e2e_steps, 5)
         hx = [x.cpu().pin_memory() for x in xs]
         hy = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
         dxb = {k: torch.empty_like(v) for k, v in bx.items()}
@@ -666,7 +761,7 @@ def run_gpu_bf16(args):
 
     if rank == 0:
         gemm_ms = float(np.mean([events[ph][0].elapsed_time(events[ph][1]) for ph in sorted(
-            {(args.warmup + s) % period for s in range(args.steps)})]))
+            {(warmup + s) % period for s in range(steps)})]))
         tot_bytes = float(sum(bf16_bytes(M, N, K, f32) for (M, N, K, f32, *_r) in calls))
         tot_flops = float(sum(2.0 * M * N * K for (M, N, K, *_r) in calls))
         peak_tf = pk["bf16_tflops_sustained"]
@@ -688,9 +783,9 @@ def run_gpu_bf16(args):
         roof["roofline_time_frac"] = round(t_roof / (gemm_ms * 1e-3), 4)
         roof["kernel"] = "gemm_bf16: " + ", ".join(sorted(set(cfgs)))
         roof["gemm_us_per_step"] = round(gemm_ms * 1000.0, 2)
-        detail = None
-        if args.detail:
-            detail = []
+        det = None
+        if detail:
+            det = []
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             for c, (M, N, K, f32, *_r) in enumerate(calls):
                 cp = wcopies[(N, K)]
@@ -711,28 +806,28 @@ def run_gpu_bf16(args):
                 us = sorted(ts)[len(ts) // 2]
                 by, fl = bf16_bytes(M, N, K, f32), 2.0 * M * N * K
                 roof_us = max(by / (pk["hbm_gbs"] * 1e3), fl / (peak_tf * 1e6))
-                detail.append({"M": M, "N": N, "K": K, "out": "f32" if f32 else "bf16", "cfg": cfgs[c],
+                det.append({"M": M, "N": N, "K": K, "out": "f32" if f32 else "bf16", "cfg": cfgs[c],
                                "us": round(us, 3), "GBps": round(by / us / 1e3, 1), "TFLOPS": round(fl / us / 1e6, 2),
                                "roofline_frac": round(roof_us / us, 3)})
-        cpu = cpu_baseline_bf16() if (args.cpu_baseline and world == 1) else None
+        cpu_line = cpu_baseline_bf16() if (cpu and world == 1) else None
         line = {
             "metric": BF16_METRIC, "value": round(step_ms * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
-            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+            "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(step_ms, 4),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x bf16 -> f32",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no dataset)",
             "config": {"workload": "bf16_small_n", "description": inputs.WORKLOADS["bf16_small_n"],
                        "calls_per_step": n_calls, "weight_rotation_mib": ROTATE_BYTES >> 20,
                        "l2": "one weight copy per use within a step; > 1 GB of activations streamed per step (L2 126 MB)",
                        "parallelism": f"replicas x{world}", "timing": "CUDA graphs replayed, CUDA events, max over ranks"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": n_calls * args.steps,
-            "clocks": clk, "dispatch": {**census, "table_hash": fb.dispatch_table_hash()}, "detail": detail,
+            "roofline": roof, "cpu_baseline": cpu_line, "e2e": e2e, "gpu_launches": n_calls * steps,
+            "clocks": clk, "dispatch": {**census, "table_hash": fb.dispatch_table_hash()}, "detail": det,
         }
-        print(json.dumps(line), flush=True)
+    else:
+        line = None
     for g in graphs:
         del g
     graphs.clear()
-    if world > 1:
-        dist.destroy_process_group()
+    return line
 
 
 def run_reference(args):
@@ -744,22 +839,25 @@ def run_reference(args):
         return run_reference_bf16(args, world)
     calls = workload_calls(args.workload)
     wcache = {}
+
+    def one(c):
+        M, N, K, i, j, o = calls[c % len(calls)]
+        m = min(M, 64)  # row-separable: large-M calls timed on 64 rows and scaled by M/64
+        x = inputs.activation_bf16(m, K, inputs.decode_seed_a(i, j), outliers=o).float().numpy()
+        return _oracle_call(x, N, K, i, wcache)[0] * M / m
+
     for s in range(args.warmup):
-        M, N, K, i, j, o = calls[s % len(calls)]
-        _oracle_call(min(M, 64), N, K, i, j, o, wcache)
-    times = []
-    for s in range(args.steps):
-        M, N, K, i, j, o = calls[(args.warmup + s) % len(calls)]
-        m = min(M, 64)
-        times.append(_oracle_call(m, N, K, i, j, o, wcache) * M / m)
+        one(s)
+    times = [one(args.warmup + s) for s in range(args.steps)]
     us = float(np.mean(times)) * 1e6
     cores = _threads()
     line = {"impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "µs/call", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1000.0, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": args.workload, "description": inputs.WORKLOADS[args.workload]},
-            "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": cores, "kind": "oracle",
-                             "sample": f"one call per step, cycling through the {args.workload} calls"},
+            "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": cores, **_host(), "kind": "oracle",
+                             "sample": f"one call per step, cycling through the {args.workload} calls; M > 64 timed "
+                                       "on 64 rows and scaled"},
             "e2e": {"value": round(us, 1), "unit": "µs/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -780,11 +878,55 @@ def run_reference_bf16(args, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1000.0, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "bf16_small_n", "description": inputs.WORKLOADS["bf16_small_n"]},
-            "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": _threads(), "kind": "oracle",
+            "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": _threads(), **_host(), "kind": "oracle",
                              "sample": "one call per step, cycling through the bf16_small_n calls; M > 64 timed on "
                                        "64 rows and scaled"},
             "e2e": {"value": round(us, 1), "unit": "µs/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+SUB_WORKLOADS = {"prefill": 5, "ladder": 3}  # steps of the extra a8w8 workloads of the default run
+BF16_SUB_STEPS = 10
+
+
+def compact(line):
+    """The fields of a workload's line that the default run carries for it."""
+    keep = ("metric", "value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config", "roofline", "quant_roofline",
+            "gpu_launches", "clocks", "dispatch", "detail", "hot")
+    return {k: line[k] for k in keep if k in line and line[k] is not None}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, dev = init_gpu()
+    try:
+        if args.workload == "bf16_small_n" and not args.shape:
+            line = measure_bf16(args, world, rank, dev, args.steps, args.warmup, args.detail, args.e2e_steps,
+                                args.cpu_baseline)
+        else:
+            line = measure_a8w8(args, world, rank, dev, args.workload, args.shape, args.steps, args.warmup,
+                                args.detail, args.e2e_steps, args.cpu_baseline)
+        torch.cuda.empty_cache()
+        if args.all_workloads and args.workload == "decode_sweep" and not args.shape:
+            # every other configuration in the same run, each as its own entry with its own
+            # roofline (bounded steps; no e2e or CPU legs)
+            subs = {}
+            for w, k in SUB_WORKLOADS.items():
+                subs[w] = measure_a8w8(args, world, rank, dev, w, None, min(args.steps, k), 3, w == "prefill", 0,
+                                       False)
+                torch.cuda.empty_cache()
+            subs["bf16_small_n"] = measure_bf16(args, world, rank, dev, min(args.steps, BF16_SUB_STEPS), 3, False, 0,
+                                                False)
+            torch.cuda.empty_cache()
+            if rank == 0:
+                line["workloads"] = {w: compact(v) for w, v in subs.items()}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
 
 
 def main():
@@ -799,13 +941,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-detail", dest="detail", action="store_false",
                     help="skip the per-shape back-to-back timing table (for profiler runs)")
+    ap.add_argument("--only", dest="all_workloads", action="store_false",
+                    help="decode sweep only: skip the prefill, ladder and bf16 entries of the default run")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
-    elif args.workload == "bf16_small_n" and not args.shape:
-        run_gpu_bf16(args)
     else:
         run_gpu(args)
 

@@ -21,7 +21,7 @@ __all__ = [
     "gemm_bf16", "workspace_bytes", "Workspace", "dispatch_lookup", "dispatch_set_row", "dispatch_reset_table",
     "dispatch_list_configs", "dispatch_stats", "dispatch_reset_stats", "dispatch_dump_json", "dispatch_table_hash",
     "get_device_status", "status_string", "version", "OP_A8W8_BLOCKSCALE", "OP_BF16", "LIB_PATH",
-    "FLAG_STATIC_WEIGHTS", "gemm_a8w8_blockscale_noalloc",
+    "FLAG_STATIC_WEIGHTS", "gemm_a8w8_blockscale_noalloc", "test_set_wait_fault",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bs.so")
@@ -63,6 +63,7 @@ _PROTOS = {
     "fp8bs_dispatch_dump_json": (_int, [ctypes.c_char_p, _sz]),
     "fp8bs_dispatch_table_hash": (_u64, []),
     "fp8bs_get_device_status": (_int, [_c_void_p]),
+    "fp8bs_test_set_wait_fault": (_int, [_u64, _i64]),
     "fp8bs_status_string": (ctypes.c_char_p, [_int]),
     "fp8bs_version": (ctypes.c_char_p, []),
 }
@@ -315,3 +316,12 @@ def dispatch_table_hash() -> str:
 def get_device_status(stream=None) -> int:
     """Synchronises the stream; returns 0 or the FP8BS_ERR_* code (6 = a device-side wait timed out)."""
     return int(lib().fp8bs_get_device_status(_stream(stream)))
+
+
+def test_set_wait_fault(wait_limit_ns: int = 0, skip_iteration: int = -1) -> None:
+    """Testing hook (fp8bs_test_set_wait_fault): bound every wait of the following
+    a8w8_tcw_* launches by wait_limit_ns (0 = the default one second) and make CTA 0's
+    producer leave K-group iteration skip_iteration unfilled (-1 = none)."""
+    st = lib().fp8bs_test_set_wait_fault(int(wait_limit_ns), int(skip_iteration))
+    if st:
+        raise Fp8bsError("fp8bs_test_set_wait_fault", st)

@@ -6,6 +6,8 @@
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -25,6 +27,19 @@ int device_sm_count() {
     counts[dev] = c;
   });
   return counts[dev];
+}
+
+int set_max_dynamic_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  if (const cudaError_t e = cudaGetDevice(&dev)) return int(e);
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count({kernel, dev})) return 0;
+  if (const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes))
+    return int(e);
+  done.insert({kernel, dev});
+  return 0;
 }
 
 bool pdl_enabled() {
@@ -61,6 +76,7 @@ static size_t op_workspace(int op, int64_t M, int64_t N, int64_t K, const Kernel
     case kPathGemvTma: return gemv_tma_workspace_bytes(M, N, K);
     case kPathGemvUmma:
       return op == FP8BS_OP_BF16 ? gemv_umma_bf16_workspace_bytes(M, N, K) : gemv_umma_workspace_bytes(M, N, K);
+    case kPathTcWide: return fp8_tc_workspace_bytes(M, N, K, cfg);
     default: return tc_workspace_bytes(op, M, N, K, cfg);
   }
 }
@@ -148,6 +164,8 @@ FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const f
   else if (cfg->path == kPathGemvUmma)
     e = launch_gemv_umma_a8w8(A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace,
                               (flags & FP8BS_FLAG_STATIC_WEIGHTS) ? 1 : 0, stream);
+  else if (cfg->path == kPathTcWide)
+    e = launch_fp8_tc(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream);
   else
     e = launch_tc_a8w8(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream);
   return from_cuda(e);
@@ -205,8 +223,15 @@ FP8BS_API fp8bs_status fp8bs_gemm_bf16(const void* A_bf16, const void* W_bf16, v
 
 FP8BS_API fp8bs_status fp8bs_get_device_status(fp8bs_stream_t stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP8BS_ERR_CUDA;
-  const unsigned int a = take_status_tc(), b = take_status_gemv_tma() | take_status_gemv_umma();
-  if (a == ~0u || b == ~0u) return FP8BS_ERR_CUDA;
-  const unsigned int v = a | b;
+  const unsigned int a = take_status_tc(), b = take_status_gemv_tma(), c = take_status_gemv_umma(),
+                     d = take_status_fp8();
+  if (a == ~0u || b == ~0u || c == ~0u || d == ~0u) return FP8BS_ERR_CUDA;
+  const unsigned int v = a | b | c | d;
   return (v & kStatusTimeout) ? FP8BS_ERR_TIMEOUT : FP8BS_OK;
+}
+
+FP8BS_API fp8bs_status fp8bs_test_set_wait_fault(uint64_t wait_limit_ns, int64_t skip_iteration) {
+  if (skip_iteration < -1 || skip_iteration > INT32_MAX) return FP8BS_ERR_INVALID_ARG;
+  fp8_tc_set_test_fault(wait_limit_ns, int(skip_iteration));
+  return FP8BS_OK;
 }

@@ -1,0 +1,478 @@
+// Tensor-core GEMM for prefill-sized M with a wide promotion epilogue: a8w8 block scale
+// on tcgen05.mma (kind::f8f6f4), TMEM accumulators, operands staged by TMA with the
+// 128-byte swizzle; persistent and warp-specialised.
+//
+//   warp 0        TMA producer: per K group one 128-row A box and one BN-row W box
+//   warp 1        TMEM allocator and MMA issuer (one thread)
+//   warps 2-3     idle (they complete warpgroup 0)
+//   warps 4..19   promotion epilogue, four warpgroups
+//
+// The block-scale definition applies a different scale to every 128-wide K group
+// ([cookbook#8]: 128x128 weight blocks, 1x128 activation groups), so a group's fp32
+// partial cannot stay in the tensor core's accumulator: every group's four K = 32 MMAs
+// write a fresh partial P_g into one of the TMEM buffers, and the epilogue reads it back
+// and adds a_scale[row, g] * w_scale[col / 128, g] * P_g into float32 registers. Reading
+// P_g back is the cost that decides the speed: 128 x BN float32 per group, against 2 x BN
+// cycles of MMA per group. Sixteen epilogue warps (each 32 TMEM lanes x BN/4 columns)
+// keep enough TMEM loads in flight to drain a buffer well inside one group's MMA time,
+// release it as soon as the data is in registers, and then scale and accumulate with
+// packed two-wide FMAs (fma.rn.f32x2, IEEE-identical to two fmaf). With BN = 256 two
+// buffers fill the 512 TMEM columns; with BN = 128 there are four.
+//
+// Split K (for shapes whose tiles leave SMs idle): a work item is (tile, K range); each
+// split stores its float32 partial tile and the last split to arrive (gpu-scope acq_rel
+// counter) sums the partials in split order -- a fixed order, so results are
+// bit-reproducible -- and rounds once to bf16.
+//
+// Every wait is bounded by a limit passed in the kernel parameters (1 s by default); a
+// wait that gives up raises the CTA's abort flag and the device status word, the roles
+// leave their loops, in-flight TMA copies and MMAs are drained (bounded) and TMEM is
+// freed before the CTA exits. For testing, the producer of CTA 0 can be told to skip one
+// K group's loads (nothing ever fills that stage, so the MMA issuer's wait runs out).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fp8bs {
+
+FP8BS_DEFINE_STATUS(fp8)
+
+constexpr int kF8Threads = 640;  // 5 warpgroups
+constexpr int kF8EpiWarps = 16;
+constexpr int kF8EpiThreads = 32 * kF8EpiWarps;
+// Registers: the launch gives every thread kF8LaunchRegs (checked by the build);
+// warpgroup 0 drops to kF8ProducerRegs and the four epilogue warpgroups rise to
+// kF8EpilogueRegs, which together use no more than the launch's 640 * kF8LaunchRegs.
+constexpr int kF8LaunchRegs = 96;
+constexpr int kF8ProducerRegs = 32;
+constexpr int kF8EpilogueRegs = 112;
+static_assert(128 * kF8ProducerRegs + kF8EpiThreads * kF8EpilogueRegs <= kF8Threads * kF8LaunchRegs, "register split");
+constexpr int kF8BM = 128;
+
+template <int BN>
+struct F8Cfg {
+  static constexpr int kABytes = kF8BM * 128;
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+  static constexpr int kBufs = 512 / BN;  // TMEM accumulators
+  static constexpr int kCols = BN / 4;    // columns per epilogue warp
+  static constexpr int kLd = 32;          // columns per TMEM load
+  static constexpr uint32_t kIdesc = make_idesc(kFmtE4M3, kFmtE4M3, kF8BM, BN);
+  static constexpr size_t kSmemBytes = size_t(kStages) * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(BN == 128 || BN == 256, "N tile");
+  static_assert(kCols % 32 == 0 && kCols % kLd == 0, "epilogue column split");
+  static_assert((2 * kStages + 2 * kBufs + 1) * 8 + 16 <= 256, "barrier region");
+};
+
+struct F8Params {
+  const float* a_scale;  // [M, G]
+  const float* w_scale;  // [ceil(N/128), G]
+  __nv_bfloat16* out;    // [M, N]
+  int M, N, G;           // G = K / 128 (K groups = K blocks)
+  int m_tiles, n_tiles;
+  int splits;            // K splits per output tile (1 = none)
+  float* part;           // splits > 1: [tiles * splits][kF8BM][BN] float32 partial tiles
+  unsigned* counter;     // splits > 1: [tiles] arrival counters (left at zero)
+  uint32_t wait_ns;            // bound of every wait (ns, below 2^32)
+  int skip_it;                 // testing: CTA 0's producer skips this K-group iteration (-1: never)
+};
+
+__device__ __forceinline__ uint32_t f8_timer() {  // low word of %globaltimer (ns; wraps every 4.3 s)
+  uint32_t t;
+  asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
+  return t;
+}
+__device__ __forceinline__ uint32_t f8_ld_flag(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void f8_st_flag(uint32_t addr) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(addr), "r"(1u) : "memory");
+}
+
+// Bounded wait with the limit of the launch (limit < 2^32 ns; differences of the low timer
+// word are exact for intervals that short). On expiry it raises the CTA's abort flag (a
+// shared-memory word) and the device status word; it also gives up once the flag is set.
+__device__ __forceinline__ bool f8_wait(uint32_t bar, uint32_t parity, uint32_t abort_addr, uint32_t limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t t0 = f8_timer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (f8_ld_flag(abort_addr)) return false;
+      if (f8_timer() - t0 > limit) {
+        f8_st_flag(abort_addr);
+        atomicOr(&g_status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Drain wait: ignores the abort flag (waits for copies or MMAs already issued), bounded.
+__device__ __forceinline__ void f8_drain(uint32_t bar, uint32_t parity, uint32_t limit) {
+  const uint32_t t0 = f8_timer();
+  while (!mbar_try_wait(bar, parity))
+    if (f8_timer() - t0 > limit) {
+      atomicOr(&g_status, kStatusTimeout);
+      return;
+    }
+}
+
+__device__ __forceinline__ void f8_epilogue_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+
+template <int kRegs>
+__device__ __forceinline__ void f8_setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs)); }
+template <int kRegs>
+__device__ __forceinline__ void f8_setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs)); }
+
+// acc[j], acc[j+1] += p0 * s, p1 * s: one packed instruction, each lane an IEEE fma (RN).
+__device__ __forceinline__ void ffma2(float& a0, float& a1, uint32_t p0, uint32_t p1, float s) {
+  unsigned long long acc, x, ss;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(acc) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(p0), "r"(p1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(x), "l"(ss));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
+}
+
+__device__ __forceinline__ uint32_t f8_pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// kCols consecutive columns of one output row as bf16, masked at M and N (N % 16 == 0,
+// so an 8-column chunk is either wholly inside or wholly outside).
+template <int kCols>
+__device__ __forceinline__ void f8_store_row(const F8Params& p, int row, int col, const float* v) {
+  if (row >= p.M) return;
+  __nv_bfloat16* dst = p.out + int64_t(row) * p.N + col;
+#pragma unroll
+  for (int j = 0; j < kCols; j += 8)
+    if (col + j < p.N)
+      *reinterpret_cast<uint4*>(dst + j) = make_uint4(f8_pack_bf16x2(v[j], v[j + 1]), f8_pack_bf16x2(v[j + 2], v[j + 3]),
+                                                      f8_pack_bf16x2(v[j + 4], v[j + 5]),
+                                                      f8_pack_bf16x2(v[j + 6], v[j + 7]));
+}
+
+// Split K: publish this split's partial tile, and if it is the last split of the tile to
+// arrive, sum the tile's partials in split order, round once and reset the counter.
+// Every epilogue thread calls this for every item (also after an abort), so the
+// epilogue barriers always see all 512 threads.
+template <int BN, int kCols>
+__device__ __forceinline__ void f8_splitk(const F8Params& p, int item, int tile, int row_in_tile, int row, int col0,
+                                          int cq, const float* acc, bool have, volatile unsigned* s_old,
+                                          volatile int* abort_flag) {
+  if (have && row < p.M) {
+    float* dst = p.part + (int64_t(item) * kF8BM + row_in_tile) * BN + cq * kCols;
+#pragma unroll
+    for (int j = 0; j < kCols; j += 4)
+      __stcg(reinterpret_cast<float4*>(dst + j), make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]));
+  }
+  f8_epilogue_bar();  // every epilogue thread's partial stores precede the release below
+  // after a timed-out wait nothing is published (the status word reports it; the caller
+  // re-zeroes the workspace before reusing it)
+  if (threadIdx.x == 128) *s_old = *abort_flag ? ~0u : atom_add_acq_rel_gpu(p.counter + tile, 1u);
+  f8_epilogue_bar();
+  if (*s_old != unsigned(p.splits - 1)) return;
+  if (row < p.M) {
+#pragma unroll 1
+    for (int c = 0; c < kCols; c += 32) {
+      float sum[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) sum[j] = 0.f;
+#pragma unroll 1
+      for (int sp = 0; sp < p.splits; ++sp) {
+        const float* src = p.part + ((int64_t(tile) * p.splits + sp) * kF8BM + row_in_tile) * BN + cq * kCols + c;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 f = __ldcg(reinterpret_cast<const float4*>(src + j));
+          sum[j] += f.x;
+          sum[j + 1] += f.y;
+          sum[j + 2] += f.z;
+          sum[j + 3] += f.w;
+        }
+      }
+      f8_store_row<32>(p, row, col0 + c, sum);
+    }
+  }
+  if (threadIdx.x == 128) p.counter[tile] = 0u;
+}
+
+template <int BN, bool kSplitK>
+__global__ void __launch_bounds__(kF8Threads, 1)
+    gemm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const F8Params p) {
+  using C = F8Cfg<BN>;
+  constexpr int S = C::kStages;
+  constexpr int NBUF = C::kBufs;
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(S) * C::kStageBytes);
+  // bars: full[S], empty[S], tfull[NBUF], tempty[NBUF], drain
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 2 * S + 2 * NBUF + 1);
+  uint32_t* tmem_slot = misc;
+  const uint32_t abort_addr = smem_u32(misc + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile unsigned* s_old = reinterpret_cast<volatile unsigned*>(misc + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + S + s); };
+  auto tfull_bar = [&](int b) { return smem_u32(bars + 2 * S + b); };
+  auto tempty_bar = [&](int b) { return smem_u32(bars + 2 * S + NBUF + b); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * S + 2 * NBUF);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < NBUF; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), kF8EpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();  // the previous kernel's results are visible from here
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int splits = kSplitK ? p.splits : 1;
+  const int items = p.m_tiles * p.n_tiles * splits;
+  const int KB = p.G;
+  const uint32_t lim = p.wait_ns;
+
+  if (warp < 4) {
+    f8_setmaxnreg_dec<kF8ProducerRegs>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      const int skip = blockIdx.x == 0 ? p.skip_it : -1;
+      int it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+        const int tile = item / splits, sp = item - tile * splits;
+        const int kb0 = KB * sp / splits, kb1 = KB * (sp + 1) / splits;
+        const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % S;
+          if (!f8_wait(empty_bar(s), ((it / S) & 1) ^ 1, abort_addr, lim)) {
+            ok = false;
+            break;
+          }
+          if (it == skip) continue;  // testing: this stage is never filled
+          const uint32_t a_dst = smem_u32(smem + size_t(s) * C::kStageBytes);
+          mbar_arrive_expect_tx(full_bar(s), C::kStageBytes);
+          tma_load_2d(a_dst, &tmA, full_bar(s), kb * 128, tm * kF8BM);
+          tma_load_2d(a_dst + C::kABytes, &tmB, full_bar(s), kb * 128, tn * BN);
+        }
+      }
+      // drain (bounded, regardless of abort): the last issue of every stage has landed.
+      // Iterations 0 .. it-1 were issued (except a skipped one, whose stage still holds
+      // the previous fill, consumed before the skip's empty wait passed).
+      for (int j = it > S ? it - S : 0; j < it; ++j)
+        if (j != skip) f8_drain(full_bar(j % S), (j / S) & 1, lim);
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      int it = 0, acc_it = 0;
+      bool ok = true, issued = false;
+      for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+        const int sp = item % splits;
+        const int kb0 = KB * sp / splits, kb1 = KB * (sp + 1) / splits;
+        for (int kb = kb0; kb < kb1; ++kb, ++it, ++acc_it) {
+          const int s = it % S;
+          const int b = acc_it % NBUF;
+          if (!f8_wait(full_bar(s), (it / S) & 1, abort_addr, lim) ||
+              !f8_wait(tempty_bar(b), ((acc_it / NBUF) & 1) ^ 1, abort_addr, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + size_t(s) * C::kStageBytes);
+          const uint64_t adesc = sw128_kmajor_desc(a_addr);
+          const uint64_t bdesc = sw128_kmajor_desc(a_addr + C::kABytes);
+          const uint32_t d_tmem = tmem_base + uint32_t(b * BN);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) umma_f8f6f4(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, C::kIdesc, kk > 0);
+          issued = true;
+          umma_commit(empty_bar(s));  // the stage is free once these MMAs have read it
+          umma_commit(tfull_bar(b));  // the group's partial is in TMEM
+        }
+      }
+      if (issued) {  // every MMA issued by this thread has completed once drain_bar flips
+        umma_commit(drain_bar);
+        f8_drain(drain_bar, 0, lim);
+      }
+    }
+  } else {
+    f8_setmaxnreg_inc<kF8EpilogueRegs>();
+    // ------------------------------------------------------------ epilogue warps 4..19
+    constexpr int kCols = C::kCols;
+    constexpr int kLd = C::kLd;
+    const int q = warp & 3;                // TMEM lane quarter this warp may access
+    const int cq = (warp - 4) >> 2;        // column quarter of the tile
+    const int row_in_tile = 32 * q + lane;
+    const uint32_t lane_addr = tmem_base + (uint32_t(32 * q) << 16) + uint32_t(cq * kCols);
+    int acc_it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < items && (kSplitK || ok); item += gridDim.x) {
+      const int tile = item / splits, sp = item - tile * splits;
+      const int kb0 = KB * sp / splits, kb1 = KB * (sp + 1) / splits;
+      const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
+      const int row = tm * kF8BM + row_in_tile;
+      const int col0 = tn * BN + cq * kCols;
+      float acc[kCols];
+#pragma unroll
+      for (int j = 0; j < kCols; ++j) acc[j] = 0.f;
+      // scales one group ahead: a_scale rows are L1 hits after the first touch
+      const int a_idx = (row < p.M ? row : 0) * KB;
+      const int w_idx = (col0 < p.N ? (col0 >> 7) : 0) * KB;
+      float sa_next = __ldg(p.a_scale + a_idx + kb0);
+      float sw_next = __ldg(p.w_scale + w_idx + kb0);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        const float sc = sa_next * sw_next;
+        if (kb + 1 < kb1) {
+          sa_next = __ldg(p.a_scale + a_idx + kb + 1);
+          sw_next = __ldg(p.w_scale + w_idx + kb + 1);
+        }
+        if (kSplitK && !ok) continue;
+        const int b = acc_it % NBUF;
+        if (!__all_sync(0xffffffffu, f8_wait(tfull_bar(b), (acc_it / NBUF) & 1, abort_addr, lim))) {
+          ok = false;
+          if (kSplitK) continue;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t t_addr = lane_addr + uint32_t(b * BN);
+#pragma unroll
+        for (int h = 0; h < kCols / kLd; ++h) {
+          uint32_t r[kLd];
+          tmem_ld_32x32b_x32(t_addr + uint32_t(kLd * h), r);
+          tmem_ld_wait();
+          if (h == kCols / kLd - 1) {  // the buffer's last columns are in registers: free it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(b));
+          }
+#pragma unroll
+          for (int j = 0; j < kLd; j += 2) ffma2(acc[kLd * h + j], acc[kLd * h + j + 1], r[j], r[j + 1], sc);
+        }
+        ++acc_it;
+      }
+      if constexpr (!kSplitK) {
+        if (!ok) break;
+        f8_store_row<kCols>(p, row, col0, acc);
+      } else {
+        f8_splitk<BN, kCols>(p, item, tile, row_in_tile, row, col0, cq, acc, ok, s_old, abort_flag);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+// Test hook: the wait bound and the skipped iteration of the next launches.
+static std::atomic<uint32_t> g_f8_wait_ns{uint32_t(kWaitLimitNs)};
+static std::atomic<int> g_f8_skip_it{-1};
+
+void fp8_tc_set_test_fault(unsigned long long wait_ns, int skip_it) {
+  // the kernel compares 32-bit timer differences: keep the bound below 2^31 ns
+  g_f8_wait_ns.store(uint32_t(wait_ns == 0 ? kWaitLimitNs : std::min<unsigned long long>(wait_ns, 2000000000ull)));
+  g_f8_skip_it.store(skip_it);
+}
+
+template <int BN, bool kSplitK>
+static int launch_f8(const void* A, const void* W, const F8Params& prm, void* stream) {
+  using C = F8Cfg<BN>;
+  if (const int e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_fp8_kernel<BN, kSplitK>),
+                                         int(C::kSmemBytes)))
+    return e;
+  CUtensorMap ma, mb;
+  if (!make_tma_2d_kmajor(&ma, A, true, prm.M, int64_t(prm.G) * 128, kF8BM) ||
+      !make_tma_2d_kmajor(&mb, W, true, prm.N, int64_t(prm.G) * 128, BN))
+    return int(cudaErrorInvalidValue);
+  const int items = prm.m_tiles * prm.n_tiles * prm.splits;
+  const int grid = std::min(items, device_sm_count());
+  return launch_kernel(gemm_fp8_kernel<BN, kSplitK>, dim3(grid), dim3(kF8Threads), C::kSmemBytes, stream, ma, mb,
+                       prm);
+}
+
+// K splits: the configuration's split_k if set, else automatic -- split only when the
+// output tiles leave most SMs idle, into enough splits to fill about one wave, at most 8
+// and at least two K groups per split.
+static int f8_splits(const KernelConfig& cfg, int64_t M, int64_t N, int64_t K) {
+  const int64_t kb = K / 128;
+  const int64_t tiles = ((M + kF8BM - 1) / kF8BM) * ((N + cfg.bn - 1) / cfg.bn);
+  int64_t sp = cfg.split_k;
+  if (sp <= 0) {
+    const int64_t sms = device_sm_count();
+    sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({(sms + tiles - 1) / tiles, kb / 2, 8});
+  }
+  sp = std::max<int64_t>(1, std::min(sp, kb));
+  if (sp > 1 && tiles > kMaxCounters) sp = 1;
+  return int(sp);
+}
+
+size_t fp8_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, const KernelConfig& cfg) {
+  const int sp = f8_splits(cfg, M, N, K);
+  if (sp == 1) return 0;
+  const int64_t tiles = ((M + kF8BM - 1) / kF8BM) * ((N + cfg.bn - 1) / cfg.bn);
+  return kCounterBytes + size_t(tiles) * sp * kF8BM * cfg.bn * sizeof(float);
+}
+
+int launch_fp8_tc(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W, const float* w_scale,
+                  void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream) {
+  // the kernel indexes the scale matrices with 32-bit integers
+  if (M * (K / 128) >= (int64_t(1) << 31) || ((N + 127) / 128) * (K / 128) >= (int64_t(1) << 31))
+    return int(cudaErrorInvalidValue);
+  F8Params p{};
+  p.a_scale = a_scale;
+  p.w_scale = w_scale;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.M = int(M);
+  p.N = int(N);
+  p.G = int(K / 128);
+  p.m_tiles = int((M + kF8BM - 1) / kF8BM);
+  p.n_tiles = int((N + cfg.bn - 1) / cfg.bn);
+  p.splits = f8_splits(cfg, M, N, K);
+  p.wait_ns = g_f8_wait_ns.load();
+  p.skip_it = g_f8_skip_it.load();
+  if (p.splits > 1) {
+    if (!ws) return int(cudaErrorInvalidValue);
+    p.counter = static_cast<unsigned*>(ws);
+    p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
+  }
+  const bool split = p.splits > 1;
+  switch (cfg.bn) {
+    case 128: return split ? launch_f8<128, true>(A, W, p, stream) : launch_f8<128, false>(A, W, p, stream);
+    case 256: return split ? launch_f8<256, true>(A, W, p, stream) : launch_f8<256, false>(A, W, p, stream);
+    default: return int(cudaErrorInvalidValue);
+  }
+}
+
+}  // namespace fp8bs

@@ -471,13 +471,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 template <bool kFp8, int BN, bool kSplitK>
 static int launch_tc_split(const void* A, const void* W, const TcParams& prm, void* stream) {
   using C = TcCfg<kFp8, BN>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_tc_kernel<kFp8, BN, kSplitK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    int(C::kSmemBytes));
-  });
-  if (attr_err != cudaSuccess) return int(attr_err);
+  if (const int attr = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_tc_kernel<kFp8, BN, kSplitK>),
+                                            int(C::kSmemBytes)))
+    return attr;
   CUtensorMap ma, mb;
   if (!make_tma_2d_kmajor(&ma, A, kFp8, prm.M, prm.K, kBM) || !make_tma_2d_kmajor(&mb, W, kFp8, prm.N, prm.K, BN))
     return int(cudaErrorInvalidValue);

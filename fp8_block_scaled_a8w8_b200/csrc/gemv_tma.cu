@@ -412,12 +412,9 @@ static int launch_gt_impl(const void* A, const float* a_scale, const void* W, co
                      int64_t N, int64_t K, void* ws, int static_w, void* stream) {
   using Cc = GtCfg<NB>;
   if ((N + kGtRows - 1) / kGtRows > kMaxCounters) return int(cudaErrorInvalidValue);
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(gemv_tma_kernel<NB, kScalesSmem>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Cc::kSmemBytes));
-  });
-  if (attr != cudaSuccess) return int(attr);
+  if (const int attr = set_max_dynamic_smem(reinterpret_cast<const void*>(gemv_tma_kernel<NB, kScalesSmem>),
+                                            int(Cc::kSmemBytes)))
+    return attr;
   CUtensorMap mw, ma;
   if (!make_tma_2d_kmajor(&mw, W, true, N, K, kGtRows) || !make_tma_2d_kmajor(&ma, A, true, M, K, 8 * NB))
     return int(cudaErrorInvalidValue);

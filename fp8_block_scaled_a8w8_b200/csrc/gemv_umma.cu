@@ -78,6 +78,12 @@ constexpr int kGuStages = 5;
 // token boxes, the activation scales) lands only once these have: fetch about what
 // the gap before the wait can absorb, not the whole ring.
 constexpr int kGuPrefetch = 4;
+// With static weights the units after those are also prefetched into L2 before the wait,
+// up to this many bytes per call over all CTAs, so the weight stream of this call runs
+// while the previous kernel finishes. The weight boxes are loaded with the evict-first L2
+// policy (they are read once), so the streaming loads of a running call do not push the
+// next call's prefetched lines out of L2.
+constexpr int64_t kGuL2PrefetchBytes = int64_t(48) << 20;
 // MMA issuing threads (lane 0 of warps 1 .. kGuIssuers): issuer i takes the units with
 // it % kGuIssuers == i. One thread spends longer issuing a unit's MMAs, waits and commits
 // than the HBM needs to deliver the unit's 16 KiB; two keep up.
@@ -105,6 +111,7 @@ struct GuParams {
   int M, N, G, nblk;
   int n_ctas;
   int static_w;          // W / w_scale are not written by any kernel still in flight
+  int l2_pre;            // static_w: units per CTA prefetched into L2 after the first kGuPrefetch
   float* part;           // [2 * n_ctas][kGuSlots][kGuRows]
   unsigned* counter;     // [nblk]
   int out_fp32;          // bf16 GEMM only
@@ -273,15 +280,25 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
       for (int s = 0; s < S; ++s) last_it[s] = -1;
       int b = first_blk, g = int(u0 - int64_t(first_blk) * G);
       int it = 0;
+      const uint64_t w_policy = l2_policy_evict_first();
       if (!kBf16 && p.static_w) {
         // The weights are not produced by an earlier kernel: fetch the first ring's worth
-        // of weight boxes before waiting for the previous kernel, overlapping its tail.
+        // of weight boxes before waiting for the previous kernel, overlapping its tail, and
+        // the next l2_pre units into L2.
         const int pre = n_units < kGuPrefetch ? n_units : kGuPrefetch;
         int pb = b, pg = g;
         for (int j = 0; j < pre; ++j) {
           const uint32_t dst = smem_u32(smem + size_t(j) * kGuStageBytes);
           mbar_arrive_expect_tx(full_bar(j), kTx);
-          tma_load_2d(dst, &tmW, full_bar(j), pg * kX, pb * kGuRows);
+          tma_load_2d_hint(dst, &tmW, full_bar(j), pg * kX, pb * kGuRows, w_policy);
+          if (++pg == G) {
+            pg = 0;
+            ++pb;
+          }
+        }
+        const int l2_end = n_units < pre + p.l2_pre ? n_units : pre + p.l2_pre;
+        for (int j = pre; j < l2_end; ++j) {
+          tma_prefetch_l2_2d(&tmW, pg * kX, pb * kGuRows);
           if (++pg == G) {
             pg = 0;
             ++pb;
@@ -305,7 +322,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
         if (!mbar_wait_bounded(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, &g_status)) break;
         const uint32_t dst = smem_u32(smem + size_t(s) * kGuStageBytes);
         mbar_arrive_expect_tx(full_bar(s), kTx);
-        tma_load_2d(dst, &tmW, full_bar(s), g * kX, b * kGuRows);
+        tma_load_2d_hint(dst, &tmW, full_bar(s), g * kX, b * kGuRows, w_policy);
         tma_load_2d(dst + kGuWBytes, &tmA, full_bar(s), g * kX, 0);
         last_it[s] = it;
         if (++g == G) {
@@ -525,16 +542,15 @@ size_t gemv_umma_bf16_workspace_bytes(int64_t, int64_t N, int64_t K) { return gu
 template <int NT, bool kBf16>
 static int launch_gu(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out, int64_t M,
                      int64_t N, int64_t K, void* ws, int static_w, int out_fp32, void* stream) {
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(gemv_umma_kernel<NT, kBf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(kGuSmemBytes));
-    if (attr == cudaSuccess)
-      attr = cudaFuncSetAttribute(gemv_umma_kernel<NT, kBf16>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                  int(cudaSharedmemCarveoutMaxShared));
+  // the carveout is a hint; the dynamic shared-memory limit is required (per device)
+  if (const int attr = set_max_dynamic_smem(reinterpret_cast<const void*>(gemv_umma_kernel<NT, kBf16>),
+                                            int(kGuSmemBytes)))
+    return attr;
+  static std::once_flag carve_once;
+  std::call_once(carve_once, [] {
+    (void)cudaFuncSetAttribute(gemv_umma_kernel<NT, kBf16>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               int(cudaSharedmemCarveoutMaxShared));
   });
-  if (attr != cudaSuccess) return int(attr);
   CUtensorMap mw, ma;
   if (!make_tma_2d_kmajor(&mw, W, !kBf16, N, K, kGuRows) || !make_tma_2d_kmajor(&ma, A, !kBf16, M, K, NT))
     return int(cudaErrorInvalidValue);
@@ -548,6 +564,11 @@ static int launch_gu(const void* A, const float* a_scale, const void* W, const f
   p.nblk = int((N + kGuRows - 1) / kGuRows);
   p.n_ctas = gu_ctas(N, K, kBf16);
   p.static_w = kBf16 ? 0 : static_w;
+  {
+    const int64_t units = int64_t(p.nblk) * p.G, per_cta = (units + p.n_ctas - 1) / p.n_ctas;
+    const int64_t budget = kGuL2PrefetchBytes / (int64_t(kGuWBytes) * p.n_ctas);
+    p.l2_pre = p.static_w ? int(std::max<int64_t>(0, std::min(per_cta, budget) - kGuPrefetch)) : 0;
+  }
   p.out_fp32 = kBf16 ? out_fp32 : 0;
   p.counter = static_cast<unsigned*>(ws);
   p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);

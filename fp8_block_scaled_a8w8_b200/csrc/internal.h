@@ -19,6 +19,7 @@ enum Path : int {
   kPathTc = 1,    // tcgen05/TMEM tensor-core kernel fed by TMA
   kPathGemvTma = 2,  // weight-streaming split-K kernel fed by TMA (mma.sync, small M)
   kPathGemvUmma = 3,  // weight-streaming split-K kernel fed by TMA, tcgen05 products (small M)
+  kPathTcWide = 4,    // tcgen05/TMEM a8w8 kernel with the sixteen-warp promotion epilogue
 };
 
 // One kernel configuration a dispatch-table row can name.
@@ -54,9 +55,13 @@ constexpr int64_t kGemvMaxM = 32;
 unsigned int take_status_tc();
 unsigned int take_status_gemv_tma();
 unsigned int take_status_gemv_umma();
+unsigned int take_status_fp8();
 
 // Device properties, cached per device.
 int device_sm_count();
+// cudaFuncAttributeMaxDynamicSharedMemorySize for a kernel, set once per (kernel, device)
+// in the context of the current device. Returns a cudaError_t value as int.
+int set_max_dynamic_smem(const void* kernel, int bytes);
 
 // ---- launchers (return a cudaError_t value as int; 0 = success) ----
 int launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q, float* scale, void* stream);
@@ -90,6 +95,13 @@ int launch_gemv_tma_noalloc(const void* A, const float* a_scale, const void* W, 
 
 // 2-D K-major TMA map, 128-byte swizzle, box = 128 bytes x box_rows.
 bool make_tma_2d_kmajor(CUtensorMap* m, const void* ptr, bool one_byte, int64_t rows, int64_t cols, int box_rows);
+
+size_t fp8_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, const KernelConfig& cfg);
+int launch_fp8_tc(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W, const float* w_scale,
+                  void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream);
+// Testing: bound of every wait (0 = the default 1 s) and an iteration whose loads CTA 0's
+// producer skips (-1 = none) for the next launches of the wide-epilogue kernel.
+void fp8_tc_set_test_fault(unsigned long long wait_ns, int skip_it);
 
 size_t tc_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, const KernelConfig& cfg);
 int launch_tc_a8w8(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W,

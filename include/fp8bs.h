@@ -21,9 +21,12 @@
  *    ("NT"): A [M,K], W [N,K], out [M,N], a_scale [M, K/128],
  *    w_scale [ceil(N/128), K/128]. Leading dimensions equal the row length
  *    unless an ld argument says otherwise.
- *  - Every pointer to matrix data is a DEVICE pointer, owned by the caller;
- *    the library never allocates, frees or retains device memory. Device
- *    pointers must be 16-byte aligned (FP8BS_ERR_ALIGNMENT otherwise).
+ *  - Every pointer to matrix data is a DEVICE pointer, owned by the caller.
+ *    The library calls no allocator: it never allocates, frees or retains
+ *    device memory (its only device storage is a few status words and the
+ *    fixed scratch array of fp8bs_gemm_a8w8_blockscale_noalloc, both part of
+ *    the library image). Device pointers must be 16-byte aligned
+ *    (FP8BS_ERR_ALIGNMENT otherwise).
  *  - Every compute call is asynchronous on the given CUDA stream (a
  *    cudaStream_t; NULL is the legacy default stream), performs no host
  *    synchronisation and no allocation, and may be captured in a CUDA graph.
@@ -34,9 +37,9 @@
  *    calls return FP8BS_ERR_CUDA or FP8BS_ERR_UNSUPPORTED.
  *  - No C++ exception crosses this interface. All functions are thread-safe;
  *    the dispatch table's counters are process-global atomics.
- *  - One device per process (one process per GPU): kernel attributes such as the
- *    dynamic shared-memory size are set once, in the context of the device that is
- *    current at a kernel's first launch.
+ *  - Calls run on the device that is current on the calling thread. Kernel
+ *    attributes such as the dynamic shared-memory size are set once per kernel
+ *    and device, at the kernel's first launch on that device.
  */
 #ifndef FP8BS_H
 #define FP8BS_H
@@ -103,8 +106,9 @@ fp8bs_status fp8bs_quant_weight_block128(const float* w_f32, int64_t N, int64_t 
  * (fp8bs_get_device_status) the workspace must be zero-filled again.
  * The kernel is picked by the dispatch table (fp8bs_dispatch_lookup): for M <= 32 a
  * weight-streaming split-K kernel (tcgen05 products, TMA-fed, stream-K over 128-row x
- * 128-column units), otherwise a tiled tcgen05/TMEM kernel fed by TMA, which also splits
- * K when its output tiles would leave most SMs idle (then it needs workspace too).
+ * 128-column units), otherwise a tiled tcgen05/TMEM kernel fed by TMA whose sixteen
+ * epilogue warps apply the block scales group by group; it also splits K when its output
+ * tiles would leave most SMs idle (then it needs workspace too).
  * Results are deterministic (split-K partial sums are reduced in a fixed order) and
  * within the float32-accumulation bound of the float64 oracle rounded once to bf16.
  */
@@ -136,7 +140,8 @@ fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const float* a_sc
  * Some callers cannot allocate device memory where they issue a GEMM -- their memory pool
  * is fixed or owned by a host framework, or an allocation there would synchronise -- so
  * they cannot supply the workspace fp8bs_gemm_a8w8_blockscale needs. This entry point
- * runs the same weight-streaming split-K kernel with its scratch taken from one fixed
+ * runs a weight-streaming split-K kernel (the TMA-fed mma.sync variant, not the tcgen05
+ * one the dispatch table picks by default) with its scratch taken from one fixed
  * 8 MiB array that is part of the library image (every GPU that loads the library holds
  * it until the process exits); it calls no allocator of any kind.
  * Arguments and result as fp8bs_gemm_a8w8_blockscale, without the workspace.
@@ -209,6 +214,22 @@ uint64_t fp8bs_dispatch_table_hash(void);
 fp8bs_status fp8bs_get_device_status(fp8bs_stream_t stream);
 
 const char* fp8bs_status_string(fp8bs_status status);
+
+/*
+ * Testing hook for the failure path of the bounded device-side waits (no counterpart in
+ * the pages; it exercises the timeout reporting of fp8bs_get_device_status). Applies to
+ * the launches that follow of the tensor-core a8w8 kernel with the wide promotion
+ * epilogue (configurations a8w8_tcw_*): every wait gives up after wait_limit_ns
+ * nanoseconds (0 restores the default of one second), and if skip_iteration >= 0 the
+ * producer of CTA 0 leaves the K-group iteration with that index (counted over the CTA's
+ * work items) unfilled, so the MMA issuer's wait on it runs out. The kernel then abandons
+ * its work, drains what it issued, frees its tensor memory and exits;
+ * fp8bs_get_device_status reports FP8BS_ERR_TIMEOUT; part of the output is not written
+ * and the workspace must be zero-filled before its next use. fp8bs_test_set_wait_fault(0,
+ * -1) restores normal operation. Process-global; not for production use.
+ * Returns FP8BS_ERR_INVALID_ARG for skip_iteration < -1 or > INT32_MAX.
+ */
+fp8bs_status fp8bs_test_set_wait_fault(uint64_t wait_limit_ns, int64_t skip_iteration);
 
 /* Library version string. */
 const char* fp8bs_version(void);

@@ -79,7 +79,7 @@ def test_c_dispatch_walk_matches_page_examples(golden_dir):
             pm, cfg = fb.dispatch_lookup(fb.OP_A8W8_BLOCKSCALE, int(m), 5120, 6144)
             assert pm == (None if want == "miss" else int(want)), (table, m, want, pm)
             if pm is None:  # a miss runs the shape's default configuration
-                assert cfg == ("a8w8_gemv_umma" if int(m) <= 32 else "a8w8_tc_bn256")
+                assert cfg == ("a8w8_gemv_umma" if int(m) <= 32 else "a8w8_tcw_bn256")
     finally:
         fb.dispatch_reset_table(keep_builtin=True)
 
@@ -111,7 +111,7 @@ def test_census_counts_and_dedup():
     assert by_m[3]["padded_M"] == 4 and by_m[3]["count"] == 3 and by_m[3]["hit"]
     assert by_m[6016]["padded_M"] == 8192
     # a miss runs the default: 1 x 4 tiles of 256 columns would leave most SMs idle, so 128
-    assert by_m[40]["hit"] is False and by_m[40]["cfg"] == "a8w8_tc_bn128"
+    assert by_m[40]["hit"] is False and by_m[40]["cfg"] == "a8w8_tcw_bn128"
     fb.dispatch_reset_stats()
     assert fb.dispatch_stats(fb.OP_A8W8_BLOCKSCALE)["hits"] == 0
 

@@ -39,7 +39,7 @@ def test_a8w8_tiled_choice(M, N, K):
     fb.dispatch_reset_table(keep_builtin=False)  # no table rows: every lookup runs the default
     try:
         _, cfg = fb.dispatch_lookup(fb.OP_A8W8_BLOCKSCALE, M, N, K)
-        assert cfg == f"a8w8_tc_bn{bn}"
+        assert cfg == f"a8w8_tcw_bn{bn}"
         sp = _splits(M, N, K, bn, K // 128)
         ws = fb.workspace_bytes(fb.OP_A8W8_BLOCKSCALE, M, N, K)
         tiles = math.ceil(M / 128) * math.ceil(N / bn)
