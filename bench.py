@@ -201,6 +201,9 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
     fb.lib()
     pk = peaks()
     calls = workload_calls(workload, shape)
+    if getattr(args, "config", None):  # force one kernel configuration (a table row per call shape)
+        for (M, N, K, *_r) in calls:
+            fb.dispatch_set_row(fb.OP_A8W8_BLOCKSCALE, M, N, K, args.config)
     uses = {}
     for (M, N, K, i, j, o) in calls:
         uses[(N, K)] = uses.get((N, K), 0) + 1
@@ -941,6 +944,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-detail", dest="detail", action="store_false",
                     help="skip the per-shape back-to-back timing table (for profiler runs)")
+    ap.add_argument("--config", default=None,
+                    help="run every a8w8 call of the workload with this kernel configuration (a dispatch row "
+                         "per call shape; names from fp8bs_dispatch_list_configs)")
     ap.add_argument("--only", dest="all_workloads", action="store_false",
                     help="decode sweep only: skip the prefill, ladder and bf16 entries of the default run")
     args = ap.parse_args()

@@ -320,7 +320,7 @@ def get_device_status(stream=None) -> int:
 
 def test_set_wait_fault(wait_limit_ns: int = 0, skip_iteration: int = -1) -> None:
     """Testing hook (fp8bs_test_set_wait_fault): bound every wait of the following
-    a8w8_tcw_* launches by wait_limit_ns (0 = the default one second) and make CTA 0's
+    a8w8_tcw_* / a8w8_tc2_* launches by wait_limit_ns (0 = the default one second) and make CTA 0's
     producer leave K-group iteration skip_iteration unfilled (-1 = none)."""
     st = lib().fp8bs_test_set_wait_fault(int(wait_limit_ns), int(skip_iteration))
     if st:

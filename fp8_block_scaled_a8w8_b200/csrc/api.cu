@@ -77,6 +77,7 @@ static size_t op_workspace(int op, int64_t M, int64_t N, int64_t K, const Kernel
     case kPathGemvUmma:
       return op == FP8BS_OP_BF16 ? gemv_umma_bf16_workspace_bytes(M, N, K) : gemv_umma_workspace_bytes(M, N, K);
     case kPathTcWide: return fp8_tc_workspace_bytes(M, N, K, cfg);
+    case kPathTcPair: return 0;
     default: return tc_workspace_bytes(op, M, N, K, cfg);
   }
 }
@@ -166,6 +167,8 @@ FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const f
                               (flags & FP8BS_FLAG_STATIC_WEIGHTS) ? 1 : 0, stream);
   else if (cfg->path == kPathTcWide)
     e = launch_fp8_tc(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream);
+  else if (cfg->path == kPathTcPair)
+    e = launch_fp8_pair(cfg->gemv_depth, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, stream);
   else
     e = launch_tc_a8w8(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream);
   return from_cuda(e);

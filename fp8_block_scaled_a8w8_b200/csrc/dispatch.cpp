@@ -34,6 +34,8 @@ static const KernelConfig kConfigs[] = {
     {"a8w8_tc_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 256, 0, 0},
     {"a8w8_tcw_bn128", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 128, 0, 0},
     {"a8w8_tcw_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 256, 0, 0},
+    {"a8w8_tc2_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcPair, 256, 1, 1},   // depth: MMA halves per K step
+    {"a8w8_tc2h_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcPair, 256, 1, 2},
     {"bf16_gemv_d2", FP8BS_OP_BF16, kPathGemv, 0, 1, 2},
     {"bf16_gemv_d4", FP8BS_OP_BF16, kPathGemv, 0, 1, 4},
     {"bf16_gemv_umma", FP8BS_OP_BF16, kPathGemvUmma, 0, 1, 0},
@@ -79,6 +81,8 @@ const KernelConfig* default_config(int op, int64_t M, int64_t N, int64_t K) {
   char nm[32];
   if (op == FP8BS_OP_A8W8_BLOCKSCALE) {
     if (M <= kGemvMaxM) return find_config(op, "a8w8_gemv_umma");
+    // (the CTA-pair configurations a8w8_tc2*_bn256 measured no faster than single CTAs
+    // with 128 x 256 tiles on the prefill shapes, so they are opt-in table rows)
     static const int fp8_bn[] = {256, 128};
     const int bn = (N % 256 == 0) ? pick_bn(M, N, fp8_bn, 2) : 128;
     std::snprintf(nm, sizeof nm, "a8w8_tcw_bn%d", bn);

@@ -78,12 +78,9 @@ constexpr int kGuStages = 5;
 // token boxes, the activation scales) lands only once these have: fetch about what
 // the gap before the wait can absorb, not the whole ring.
 constexpr int kGuPrefetch = 4;
-// With static weights the units after those are also prefetched into L2 before the wait,
-// up to this many bytes per call over all CTAs, so the weight stream of this call runs
-// while the previous kernel finishes. The weight boxes are loaded with the evict-first L2
-// policy (they are read once), so the streaming loads of a running call do not push the
-// next call's prefetched lines out of L2.
-constexpr int64_t kGuL2PrefetchBytes = int64_t(48) << 20;
+// (An L2 prefetch of the following units before the wait was measured: it made N = 5120
+// and N = 14336 calls 5% slower and N = 34816 calls no faster, so it is not done.)
+// The weight boxes are loaded with the evict-first L2 policy: they are read once per call.
 // MMA issuing threads (lane 0 of warps 1 .. kGuIssuers): issuer i takes the units with
 // it % kGuIssuers == i. One thread spends longer issuing a unit's MMAs, waits and commits
 // than the HBM needs to deliver the unit's 16 KiB; two keep up.
@@ -111,7 +108,6 @@ struct GuParams {
   int M, N, G, nblk;
   int n_ctas;
   int static_w;          // W / w_scale are not written by any kernel still in flight
-  int l2_pre;            // static_w: units per CTA prefetched into L2 after the first kGuPrefetch
   float* part;           // [2 * n_ctas][kGuSlots][kGuRows]
   unsigned* counter;     // [nblk]
   int out_fp32;          // bf16 GEMM only
@@ -283,22 +279,13 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
       const uint64_t w_policy = l2_policy_evict_first();
       if (!kBf16 && p.static_w) {
         // The weights are not produced by an earlier kernel: fetch the first ring's worth
-        // of weight boxes before waiting for the previous kernel, overlapping its tail, and
-        // the next l2_pre units into L2.
+        // of weight boxes before waiting for the previous kernel, overlapping its tail.
         const int pre = n_units < kGuPrefetch ? n_units : kGuPrefetch;
         int pb = b, pg = g;
         for (int j = 0; j < pre; ++j) {
           const uint32_t dst = smem_u32(smem + size_t(j) * kGuStageBytes);
           mbar_arrive_expect_tx(full_bar(j), kTx);
           tma_load_2d_hint(dst, &tmW, full_bar(j), pg * kX, pb * kGuRows, w_policy);
-          if (++pg == G) {
-            pg = 0;
-            ++pb;
-          }
-        }
-        const int l2_end = n_units < pre + p.l2_pre ? n_units : pre + p.l2_pre;
-        for (int j = pre; j < l2_end; ++j) {
-          tma_prefetch_l2_2d(&tmW, pg * kX, pb * kGuRows);
           if (++pg == G) {
             pg = 0;
             ++pb;
@@ -564,11 +551,6 @@ static int launch_gu(const void* A, const float* a_scale, const void* W, const f
   p.nblk = int((N + kGuRows - 1) / kGuRows);
   p.n_ctas = gu_ctas(N, K, kBf16);
   p.static_w = kBf16 ? 0 : static_w;
-  {
-    const int64_t units = int64_t(p.nblk) * p.G, per_cta = (units + p.n_ctas - 1) / p.n_ctas;
-    const int64_t budget = kGuL2PrefetchBytes / (int64_t(kGuWBytes) * p.n_ctas);
-    p.l2_pre = p.static_w ? int(std::max<int64_t>(0, std::min(per_cta, budget) - kGuPrefetch)) : 0;
-  }
   p.out_fp32 = kBf16 ? out_fp32 : 0;
   p.counter = static_cast<unsigned*>(ws);
   p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);

@@ -20,6 +20,7 @@ enum Path : int {
   kPathGemvTma = 2,  // weight-streaming split-K kernel fed by TMA (mma.sync, small M)
   kPathGemvUmma = 3,  // weight-streaming split-K kernel fed by TMA, tcgen05 products (small M)
   kPathTcWide = 4,    // tcgen05/TMEM a8w8 kernel with the sixteen-warp promotion epilogue
+  kPathTcPair = 5,    // the same on CTA pairs (cta_group::2, 256 x 256 tiles)
 };
 
 // One kernel configuration a dispatch-table row can name.
@@ -29,7 +30,7 @@ struct KernelConfig {
   int path;         // Path
   int bn;           // tensor-core path: N tile (columns of W per CTA)
   int split_k;      // tensor-core path: K splits (0 = automatic from the tile count, 1 = none)
-  int gemv_depth;   // weight-streaming path: units in flight per warp
+  int gemv_depth;   // weight-streaming path: units in flight per warp; CTA-pair path: MMAs per K step
 };
 
 // Registry of every configuration (static storage).
@@ -95,10 +96,16 @@ int launch_gemv_tma_noalloc(const void* A, const float* a_scale, const void* W, 
 
 // 2-D K-major TMA map, 128-byte swizzle, box = 128 bytes x box_rows.
 bool make_tma_2d_kmajor(CUtensorMap* m, const void* ptr, bool one_byte, int64_t rows, int64_t cols, int box_rows);
+// 2-D bf16 [rows, cols] map for TMA stores: box 32 x 32, 64-byte swizzle.
+bool make_tma_2d_bf16_store(CUtensorMap* m, void* ptr, int64_t rows, int64_t cols);
 
 size_t fp8_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, const KernelConfig& cfg);
 int launch_fp8_tc(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W, const float* w_scale,
                   void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream);
+// CTA-pair kernel (no split K, no workspace) and the clusters of two that fit at once.
+int launch_fp8_pair(int halves, const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
+                    int64_t M, int64_t N, int64_t K, void* stream);
+int fp8_pair_clusters();
 // Testing: bound of every wait (0 = the default 1 s) and an iteration whose loads CTA 0's
 // producer skips (-1 = none) for the next launches of the wide-epilogue kernel.
 void fp8_tc_set_test_fault(unsigned long long wait_ns, int skip_it);

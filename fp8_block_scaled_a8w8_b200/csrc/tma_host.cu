@@ -40,4 +40,20 @@ bool make_tma_2d_kmajor(CUtensorMap* m, const void* ptr, bool one_byte, int64_t 
   return r == CUDA_SUCCESS;
 }
 
+// 2-D map over a row-major bf16 [rows, cols] output for TMA stores: box = 32 columns (64
+// bytes) x 32 rows, 64-byte swizzle (the layout the epilogue stages in shared memory);
+// elements outside [rows, cols] are not written.
+bool make_tma_2d_bf16_store(CUtensorMap* m, void* ptr, int64_t rows, int64_t cols) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(cols * 2)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  std::memset(m, 0, sizeof(*m));
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace fp8bs

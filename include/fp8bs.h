@@ -107,8 +107,10 @@ fp8bs_status fp8bs_quant_weight_block128(const float* w_f32, int64_t N, int64_t 
  * The kernel is picked by the dispatch table (fp8bs_dispatch_lookup): for M <= 32 a
  * weight-streaming split-K kernel (tcgen05 products, TMA-fed, stream-K over 128-row x
  * 128-column units), otherwise a tiled tcgen05/TMEM kernel fed by TMA whose sixteen
- * epilogue warps apply the block scales group by group; it also splits K when its output
- * tiles would leave most SMs idle (then it needs workspace too).
+ * epilogue warps apply the block scales group by group and store the output through
+ * shared memory with TMA; it also splits K when its output tiles would leave most SMs
+ * idle (then the call needs workspace too). A table row may instead name the CTA-pair
+ * variant (tcgen05 cta_group::2, 256 x 256 tiles, configurations a8w8_tc2*).
  * Results are deterministic (split-K partial sums are reduced in a fixed order) and
  * within the float32-accumulation bound of the float64 oracle rounded once to bf16.
  */
@@ -218,11 +220,12 @@ const char* fp8bs_status_string(fp8bs_status status);
 /*
  * Testing hook for the failure path of the bounded device-side waits (no counterpart in
  * the pages; it exercises the timeout reporting of fp8bs_get_device_status). Applies to
- * the launches that follow of the tensor-core a8w8 kernel with the wide promotion
- * epilogue (configurations a8w8_tcw_*): every wait gives up after wait_limit_ns
+ * the launches that follow of the tensor-core a8w8 kernels with the wide promotion
+ * epilogue (configurations a8w8_tcw_* and a8w8_tc2_*): every wait gives up after wait_limit_ns
  * nanoseconds (0 restores the default of one second), and if skip_iteration >= 0 the
  * producer of CTA 0 leaves the K-group iteration with that index (counted over the CTA's
- * work items) unfilled, so the MMA issuer's wait on it runs out. The kernel then abandons
+ * work items) unfilled, so the MMA issuer's wait on it runs out (for CTA pairs, the
+ * other waits of the pair then run out too). The kernel then abandons
  * its work, drains what it issued, frees its tensor memory and exits;
  * fp8bs_get_device_status reports FP8BS_ERR_TIMEOUT; part of the output is not written
  * and the workspace must be zero-filled before its next use. fp8bs_test_set_wait_fault(0,

@@ -2,9 +2,9 @@
 
 Restates the documented policy in Python and checks the library's choices against it:
 M <= 32 runs the weight-streaming kernel; otherwise the tiled kernel takes the widest tile
-whose output tiles give at least half of the SMs a tile, and splits K (workspace > 0) only
-when even the narrowest tile leaves that many SMs idle. Without a GPU the library assumes
-148 SMs (B200).
+whose output tiles give at least half of the SMs a tile, and splits K (workspace > 0)
+only when even the narrowest tile leaves that many SMs idle. Without a
+GPU the library assumes 148 SMs (B200).
 """
 
 import math

@@ -88,7 +88,8 @@ def test_tc_path_parity(M, N, K):
     check_a8w8(_run(*case), *case)
 
 
-@pytest.mark.parametrize("cfg", ["a8w8_tc_bn128", "a8w8_tc_bn256", "a8w8_tcw_bn128", "a8w8_tcw_bn256"])
+@pytest.mark.parametrize("cfg", ["a8w8_tc_bn128", "a8w8_tc_bn256", "a8w8_tcw_bn128", "a8w8_tcw_bn256",
+                                 "a8w8_tc2_bn256", "a8w8_tc2h_bn256"])
 @pytest.mark.parametrize("M,N,K", [(1, 256, 128), (40, 512, 2048), (300, 1536, 640), (2, 272, 256),
                                    (1000, 2560, 1024), (777, 4112, 768)])
 def test_tc_configs_any_m(cfg, M, N, K):
@@ -100,7 +101,9 @@ def test_tc_configs_any_m(cfg, M, N, K):
 @pytest.mark.parametrize("M,N,K,cfg", [(3, 272, 512, None), (16, 1024, 1024, None), (200, 512, 1024, None),
                                        (130, 384, 512, "a8w8_tc_bn128"), (64, 512, 384, "a8w8_tc_bn256"),
                                        (130, 384, 512, "a8w8_tcw_bn128"), (64, 512, 384, "a8w8_tcw_bn256"),
-                                       (1100, 2816, 1024, "a8w8_tcw_bn256")])
+                                       (1100, 2816, 1024, "a8w8_tcw_bn256"), (300, 272, 512, "a8w8_tc2_bn256"),
+                                       (2100, 4864, 1024, "a8w8_tc2_bn256"), (300, 272, 512, "a8w8_tc2h_bn256"),
+                                       (2100, 4864, 1024, "a8w8_tc2h_bn256")])
 def test_integer_valued_bit_exact(M, N, K, cfg):
     """Integer e4m3 values |v| <= 4 and power-of-two scales: every partial sum is exact,
     so the bf16 output must equal bf16(exact) bit for bit."""
@@ -115,7 +118,8 @@ def test_integer_valued_bit_exact(M, N, K, cfg):
     assert np.array_equal(y.float().cpu().numpy().astype(np.float64), ref_bf16)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 5120, 6144), (9, 2048, 1024), (700, 1024, 1024), (2100, 5120, 1024)])
+@pytest.mark.parametrize("M,N,K", [(1, 5120, 6144), (9, 2048, 1024), (700, 1024, 1024), (2100, 5120, 1024),
+                                   (4100, 9728, 1024)])
 def test_deterministic_and_graph_replay(M, N, K):
     case = _raw_case(M, N, K, seed=3)
     A, a_s, W, w_s = (codes_to_device(case[0]), torch.from_numpy(case[1]).cuda(), codes_to_device(case[2]),

@@ -1,8 +1,9 @@
 """The failure path of the bounded device-side waits, made to run without any fault.
 
 The testing hook fp8bs_test_set_wait_fault shortens every wait of the tensor-core a8w8
-kernel (configurations a8w8_tcw_*) to 20 ms and has CTA 0's producer leave one K group's
-stage unfilled, so the MMA issuer's wait on that stage runs out. The kernel must give up,
+kernels (configurations a8w8_tcw_* and the CTA-pair a8w8_tc2_*) to 20 ms and has CTA 0's
+producer leave one K group's stage unfilled, so the MMA issuer's wait on that stage runs
+out (with CTA pairs the peer's waits then run out on their own). The kernel must give up,
 drain what it issued, free its tensor memory and return; the host then reads
 FP8BS_ERR_TIMEOUT from fp8bs_get_device_status, and the next call -- on a re-zeroed
 workspace, with the hook cleared -- must be correct against the oracle.
@@ -27,6 +28,9 @@ TIMEOUT = 6  # FP8BS_ERR_TIMEOUT
     (1024, 2560, 1024, "a8w8_tcw_bn256", 3),   # 80 tiles, no split K
     (256, 1024, 2048, "a8w8_tcw_bn128", 1),    # 16 tiles x 8 K splits
     (1000, 2560, 1024, "a8w8_tcw_bn128", 0),   # the very first stage
+    (2048, 4864, 1024, "a8w8_tc2_bn256", 3),   # CTA pairs: the leader's stage 3
+    (300, 512, 512, "a8w8_tc2_bn256", 0),      # CTA pairs, a single pair tile
+    (2048, 4864, 1024, "a8w8_tc2h_bn256", 5),  # CTA pairs, two MMA halves per K step
 ])
 def test_wait_runs_out_reports_timeout_and_recovers(M, N, K, cfg, skip):
     A_q = inputs.random_e4m3_codes((M, K), 1)
