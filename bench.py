@@ -19,8 +19,9 @@ the step time is the max over ranks. N>1 runs N independent replicas (the path
 has no exchange step).
 
 The default run also measures, with a few steps each, every other configuration: the
-prefill shapes, the dense M ladder (with the dispatch census and its padded-M drift) and
-the bf16 small-N GEMMs, each as an entry of "workloads" with its own roofline; the
+prefill shapes, the dense M ladder (with the dispatch census and its padded-M drift), the
+bf16 small-N GEMMs and the bf16 lm_head, each as an entry of "workloads" with its own
+roofline; the
 per-shape "detail" table gives cold- and hot-weight us/call, and the CPU leg reports the
 oracle's time and the accuracy of the timed outputs against it. --only skips the extra
 workloads.
@@ -607,11 +608,17 @@ def cpu_baseline(workload, calls=None, xs=None, gpu_output=None, budget_s=20.0):
 
 
 # --------------------------------------------------------------------------- bf16 small-N workload
-BF16_METRIC = "bf16 small-N GEMM µs/call, TFLOPS & HBM GB/s (cold weights) vs roofline"
+BF16_METRIC = "bf16 GEMM µs/call, TFLOPS & HBM GB/s (cold weights) vs roofline"
 
 
-def bf16_calls():
-    """(M, N, K, out_fp32, nk_index, m_index) of the small-N BF16 workload."""
+BF16_WORKLOADS = ("bf16_small_n", "lm_head")
+
+
+def bf16_calls(workload="bf16_small_n"):
+    """(M, N, K, out_fp32, nk_index, m_index) of a bf16 workload."""
+    if workload == "lm_head":
+        N, K = inputs.LM_HEAD_NK
+        return [(M, N, K, False, 0, j) for j, M in enumerate(inputs.LM_HEAD_MS)]
     return [(M, N, K, f32, i, j) for i, (N, K, f32) in enumerate(inputs.BF16_NK) for j, M in enumerate(inputs.BF16_MS)]
 
 
@@ -625,8 +632,8 @@ def _oracle_bf16_call(M, N, K, f32, i, j, wcache):
     return time.perf_counter() - t0
 
 
-def cpu_baseline_bf16(budget_s=20.0):
-    calls = bf16_calls()
+def cpu_baseline_bf16(workload="bf16_small_n", budget_s=20.0):
+    calls = bf16_calls(workload)
     order = list(np.random.default_rng(0).permutation(len(calls)))
     wcache, spent, done = {}, 0.0, []
     for c in order:
@@ -639,12 +646,12 @@ def cpu_baseline_bf16(budget_s=20.0):
             break
     return {"value": round(float(np.mean(done)) * 1e6, 1), "unit": "µs/call", "cores": _threads(), **_host(),
             "kind": "oracle",
-            "sample": f"{len(done)} of {len(calls)} calls of the bf16_small_n workload (random order), float64 "
+            "sample": f"{len(done)} of {len(calls)} calls of the {workload} workload (random order), float64 "
                       "matmul; calls with M > 64 timed on 64 rows and scaled by M/64"}
 
 
-def measure_bf16(args, world, rank, dev, steps, warmup, detail, e2e_steps, cpu):
-    """The JSON line of the bf16 small-N workload (rank 0; None elsewhere)."""
+def measure_bf16(args, world, rank, dev, steps, warmup, detail, e2e_steps, cpu, workload="bf16_small_n"):
+    """The JSON line of a bf16 workload (rank 0; None elsewhere)."""
     import torch
     import torch.distributed as dist
 
@@ -652,7 +659,7 @@ def measure_bf16(args, world, rank, dev, steps, warmup, detail, e2e_steps, cpu):
 
     fb.lib()
     pk = peaks()
-    calls = bf16_calls()
+    calls = bf16_calls(workload)
     n_calls = len(calls)
     uses, maxm = {}, {}
     for (M, N, K, f32, i, j) in calls:
@@ -812,13 +819,13 @@ def measure_bf16(args, world, rank, dev, steps, warmup, detail, e2e_steps, cpu):
                 det.append({"M": M, "N": N, "K": K, "out": "f32" if f32 else "bf16", "cfg": cfgs[c],
                                "us": round(us, 3), "GBps": round(by / us / 1e3, 1), "TFLOPS": round(fl / us / 1e6, 2),
                                "roofline_frac": round(roof_us / us, 3)})
-        cpu_line = cpu_baseline_bf16() if (cpu and world == 1) else None
+        cpu_line = cpu_baseline_bf16(workload) if (cpu and world == 1) else None
         line = {
             "metric": BF16_METRIC, "value": round(step_ms * 1000.0 / (n_calls * world), 3), "unit": "µs/call",
             "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": round(step_ms, 4),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16 x bf16 -> f32",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights; no dataset)",
-            "config": {"workload": "bf16_small_n", "description": inputs.WORKLOADS["bf16_small_n"],
+            "config": {"workload": workload, "description": inputs.WORKLOADS[workload],
                        "calls_per_step": n_calls, "weight_rotation_mib": ROTATE_BYTES >> 20,
                        "l2": "one weight copy per use within a step; > 1 GB of activations streamed per step (L2 126 MB)",
                        "parallelism": f"replicas x{world}", "timing": "CUDA graphs replayed, CUDA events, max over ranks"},
@@ -838,7 +845,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if world > 1 and rank != 0:
         return
-    if args.workload == "bf16_small_n":
+    if args.workload in BF16_WORKLOADS:
         return run_reference_bf16(args, world)
     calls = workload_calls(args.workload)
     wcache = {}
@@ -866,7 +873,7 @@ def run_reference(args):
 
 
 def run_reference_bf16(args, world):
-    calls = bf16_calls()
+    calls = bf16_calls(args.workload)
     wcache = {}
     for s in range(args.warmup):
         M, N, K, f32, i, j = calls[s % len(calls)]
@@ -880,9 +887,9 @@ def run_reference_bf16(args, world):
     line = {"impl": "reference", "metric": BF16_METRIC, "value": round(us, 1), "unit": "µs/call", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1000.0, 3), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "bf16_small_n", "description": inputs.WORKLOADS["bf16_small_n"]},
+            "config": {"workload": args.workload, "description": inputs.WORKLOADS[args.workload]},
             "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": _threads(), **_host(), "kind": "oracle",
-                             "sample": "one call per step, cycling through the bf16_small_n calls; M > 64 timed on "
+                             "sample": f"one call per step, cycling through the {args.workload} calls; M > 64 timed on "
                                        "64 rows and scaled"},
             "e2e": {"value": round(us, 1), "unit": "µs/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -905,9 +912,9 @@ def run_gpu(args):
 
     world, rank, dev = init_gpu()
     try:
-        if args.workload == "bf16_small_n" and not args.shape:
+        if args.workload in BF16_WORKLOADS and not args.shape:
             line = measure_bf16(args, world, rank, dev, args.steps, args.warmup, args.detail, args.e2e_steps,
-                                args.cpu_baseline)
+                                args.cpu_baseline, args.workload)
         else:
             line = measure_a8w8(args, world, rank, dev, args.workload, args.shape, args.steps, args.warmup,
                                 args.detail, args.e2e_steps, args.cpu_baseline)
@@ -920,9 +927,10 @@ def run_gpu(args):
                 subs[w] = measure_a8w8(args, world, rank, dev, w, None, min(args.steps, k), 3, w == "prefill", 0,
                                        False)
                 torch.cuda.empty_cache()
-            subs["bf16_small_n"] = measure_bf16(args, world, rank, dev, min(args.steps, BF16_SUB_STEPS), 3, False, 0,
-                                                False)
-            torch.cuda.empty_cache()
+            for w in BF16_WORKLOADS:
+                subs[w] = measure_bf16(args, world, rank, dev, min(args.steps, BF16_SUB_STEPS), 3, w == "lm_head", 0,
+                                       False, w)
+                torch.cuda.empty_cache()
             if rank == 0:
                 line["workloads"] = {w: compact(v) for w, v in subs.items()}
         if rank == 0:

@@ -89,11 +89,18 @@ const KernelConfig* default_config(int op, int64_t M, int64_t N, int64_t K) {
     return find_config(op, nm);
   }
   if (M <= kGemvMaxM) return find_config(op, "bf16_gemv_umma");
-  // widest first among the widths that tile N without a ragged last tile, then narrower
+  // widest first among the widths that tile N without a ragged last tile, then narrower;
+  // a large N (an lm_head) takes 256 or 128 even with a ragged last tile, which costs
+  // less than re-reading A for every narrow tile
   static const int all_bn[] = {256, 192, 128, 64, 32};
   int cands[5], n = 0;
-  for (int b : all_bn)
-    if (b <= N && N % b == 0) cands[n++] = b;
+  if (N >= 2048) {
+    cands[n++] = 256;
+    cands[n++] = 128;
+  } else {
+    for (int b : all_bn)
+      if (b <= N && N % b == 0) cands[n++] = b;
+  }
   if (n == 0) cands[n++] = 32;
   if (N < 256 && N % 32 == 0 && N != cands[0]) {  // a single tile as wide as N comes first
     for (int i = n; i > 0; --i) cands[i] = cands[i - 1];
@@ -136,6 +143,8 @@ void add_builtin_rows(std::map<Key, const KernelConfig*>& rows) {
   const int64_t bms[] = {1, 32, 576, 4096, 16384};
   for (const auto& p : bnk)
     for (int64_t m : bms) rows[Key{FP8BS_OP_BF16, m, p[0], p[1]}] = default_config(FP8BS_OP_BF16, m, p[0], p[1]);
+  for (int64_t m : {32, 512, 1024, 2048, 4096})  // lm_head (N = 32320, K = 5120) at the power-of-two ladder
+    rows[Key{FP8BS_OP_BF16, m, 32320, 5120}] = default_config(FP8BS_OP_BF16, m, 32320, 5120);
 }
 
 State& state() {

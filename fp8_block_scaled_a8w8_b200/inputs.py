@@ -34,6 +34,9 @@ LADDER_NK = (5120, 6144)
 # small-N bf16 GEMMs: (N, K, fp32 output?)
 BF16_NK = [(256, 6144, False), (32, 6144, False), (384, 5120, False), (1024, 5120, True), (128, 512, False)]
 BF16_MS = [1, 32, 576, 4096, 16384]
+# the target lm_head of [aiter#7247] "Technical Details" / microbenchmark table (bf16 out)
+LM_HEAD_NK = (32320, 5120)
+LM_HEAD_MS = [24, 384, 1536, 2304, 3072]
 
 WORKLOADS = {
     "decode_m1_n5120_k6144": "single a8w8 blockscale GEMM M=1, N=5120, K=6144, seed 0",
@@ -44,6 +47,7 @@ WORKLOADS = {
     "ladder": "a8w8 blockscale dense M ladder, 512 M drawn from 1..8192 on (N,K)=(5120,6144)",
     "bf16_small_n": "bf16 x bf16 small-N GEMMs, M in {1,32,576,4096,16384} x (N,K) in "
                     "{(256,6144),(32,6144),(384,5120),(1024,5120) fp32 out,(128,512)}",
+    "lm_head": "bf16 x bf16 large-N lm_head GEMM, M in {24,384,1536,2304,3072} on (N,K)=(32320,5120), bf16 out",
 }
 
 

@@ -62,3 +62,25 @@ def test_bf16_full_size_sampled_rows(M, N, K, out_fp32):
     y, A, W = _run(M, N, K, out_fp32, seed=9)
     rows = np.unique(np.concatenate([[0, 127, 128, M - 1], np.random.default_rng(M).choice(M, 12, replace=False)]))
     check_bf16(y, A, W, out_fp32, rows=rows)
+
+
+_LM = {}
+
+
+@pytest.mark.parametrize("M", inputs.LM_HEAD_MS)
+def test_lm_head_full_size_sampled_rows(M):
+    """The large-N bf16 lm_head (N = 32320, K = 5120: the last 256-column tile is ragged)
+    at the M values the pages measure, on 48 rows: first and last rows, both sides of
+    128-row tile boundaries, seeded random rows."""
+    N, K = inputs.LM_HEAD_NK
+    if "W" not in _LM:
+        _LM["W"] = inputs.weight_bf16(N, K, 41)
+        _LM["Wd"] = _LM["W"].cuda()
+    A = inputs.activation_bf16(M, K, 42 + M)
+    y = fb.gemm_bf16(A.cuda(), _LM["Wd"])
+    torch.cuda.synchronize()
+    assert fb.get_device_status() == 0
+    rng = np.random.default_rng(M)
+    fixed = [0, 1, M - 1] + [t for b in range(128, M, 128) for t in (b - 1, b)][:16]
+    rows = np.unique(np.concatenate([fixed, rng.choice(M, min(M, 48 - len(fixed)), replace=False)]))
+    check_bf16(y, A.float().numpy(), _LM["W"].float().numpy(), False, rows=rows)

@@ -48,10 +48,14 @@ def test_a8w8_tiled_choice(M, N, K):
         fb.dispatch_reset_table(keep_builtin=True)
 
 
-@pytest.mark.parametrize("M", [576, 4096, 16384, 40, 200])
-@pytest.mark.parametrize("N,K", [(256, 6144), (32, 6144), (384, 5120), (1024, 5120), (128, 512), (48, 192)])
+@pytest.mark.parametrize("M", [576, 4096, 16384, 40, 200, 24 + 16, 3072])
+@pytest.mark.parametrize("N,K", [(256, 6144), (32, 6144), (384, 5120), (1024, 5120), (128, 512), (48, 192),
+                                 (32320, 5120), (2064, 1024)])
 def test_bf16_tiled_choice(M, N, K):
-    cands = [b for b in (256, 192, 128, 64, 32) if b <= N and N % b == 0] or [32]
+    if N >= 2048:  # large N: 256 or 128 even with a ragged last tile
+        cands = [256, 128]
+    else:
+        cands = [b for b in (256, 192, 128, 64, 32) if b <= N and N % b == 0] or [32]
     if N < 256 and N % 32 == 0 and N != cands[0]:
         cands = [N] + cands
     bn = _pick(M, N, cands)
