@@ -20,8 +20,8 @@ has no exchange step).
 
 The default run also measures, with a few steps each, every other configuration: the
 prefill shapes, the dense M ladder (with the dispatch census and its padded-M drift), the
-bf16 small-N GEMMs and the bf16 lm_head, each as an entry of "workloads" with its own
-roofline; the
+bf16 small-N GEMMs, the bf16 lm_head and the fused residual add + RMSNorm + quantisation
+step, each as an entry of "workloads" with its own roofline; the
 per-shape "detail" table gives cold- and hot-weight us/call, and the CPU leg reports the
 oracle's time and the accuracy of the timed outputs against it. --only skips the extra
 workloads.
@@ -840,6 +840,103 @@ def measure_bf16(args, world, rank, dev, steps, warmup, detail, e2e_steps, cpu, 
     return line
 
 
+# --------------------------------------------------------------------------- fused norm + quant workload
+NORM_METRIC = "add_rmsnorm_quant µs/call & HBM GB/s vs roofline"
+
+
+def norm_bytes(M, K):
+    """x + residual read, residual_out written (bf16), codes written, scales written, gamma read."""
+    return 7 * M * K + 4 * M * (K // 128) + 2 * K
+
+
+def measure_norm(args, world, rank, dev, steps, warmup):
+    """The fused residual add + RMSNorm + activation quantisation over the decode and prefill
+    token counts (rank 0's line; None elsewhere)."""
+    import torch
+
+    import fp8_block_scaled_a8w8_b200 as fb
+
+    fb.lib()
+    pk = peaks()
+    calls = [(M, K) for K in inputs.NORM_KS for M in inputs.NORM_MS]
+    bufs = []
+    for i, (M, K) in enumerate(calls):
+        x = inputs.activation_bf16(M, K, 300 + i).to(dev)
+        r = inputs.activation_bf16(M, K, 400 + i).to(dev)
+        g = (1.0 + 0.1 * inputs.activation_bf16(1, K, 500 + i).float()).to(torch.bfloat16)[0].to(dev)
+        bufs.append((x, r, g, torch.empty_like(x), torch.empty((M, K), dtype=torch.float8_e4m3fn, device=dev),
+                     torch.empty((M, K // 128), dtype=torch.float32, device=dev)))
+    stream = torch.cuda.Stream(device=dev)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        for (x, r, g, ro, q, s) in bufs:
+            fb.add_rmsnorm_quant(x, r, g, 1e-6, residual_out=ro, q=q, scale=s, stream=stream)
+        if e is not None:
+            e[1].record(stream)
+
+    with torch.cuda.stream(stream):
+        step()
+        stream.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            step(ev)
+        for _ in range(warmup):
+            graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index)
+    if rank == 0:
+        clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(steps):
+        with torch.cuda.stream(stream):
+            graph.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop() if rank == 0 else None
+    step_ms = max_over_ranks(t0.elapsed_time(t1) / steps, dev)
+    line = None
+    if rank == 0:
+        tot = float(sum(norm_bytes(M, K) for M, K in calls))
+        ms = ev[0].elapsed_time(ev[1])
+        ach = tot / (ms * 1e-3) / 1e9
+        detail = []
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for (M, K), (x, r, g, ro, q, s) in zip(calls, bufs):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                with torch.cuda.graph(gr, stream=stream):
+                    for _ in range(20):
+                        fb.add_rmsnorm_quant(x, r, g, 1e-6, residual_out=ro, q=q, scale=s, stream=stream)
+                ts = []
+                for _ in range(5):
+                    e0.record(stream)
+                    gr.replay()
+                    e1.record(stream)
+                    e1.synchronize()
+                    ts.append(e0.elapsed_time(e1) * 1000.0 / 20)
+            del gr
+            us = sorted(ts)[len(ts) // 2]
+            detail.append({"M": M, "K": K, "us": round(us, 3), "GBps": round(norm_bytes(M, K) / us / 1e3, 1),
+                           "roofline_frac": round(norm_bytes(M, K) / (pk["hbm_gbs"] * 1e3) / us, 3),
+                           "note": "20 back-to-back calls on the same buffers (hot in L2 when they fit)"})
+        line = {"metric": NORM_METRIC, "value": round(step_ms * 1000.0 / (len(calls) * world), 3), "unit": "µs/call",
+                "ms_per_step": round(step_ms, 4), "steps": steps, "warmup": warmup, "dtype": "bf16 -> f32 -> e4m3",
+                "config": {"workload": "add_rmsnorm_quant", "description": inputs.WORKLOADS["add_rmsnorm_quant"],
+                           "calls_per_step": len(calls),
+                           "l2": f"{tot / 1e6:.0f} MB moved per step (> 126 MB L2)"},
+                "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": round(ach / pk["hbm_gbs"], 4), "traffic": None,
+                             "kernel": "add_rmsnorm_quant_kernel", "algorithmic_bytes_per_step": int(tot)},
+                "gpu_launches": len(calls) * steps, "clocks": clk, "detail": detail}
+    del graph
+    return line
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -847,6 +944,8 @@ def run_reference(args):
         return
     if args.workload in BF16_WORKLOADS:
         return run_reference_bf16(args, world)
+    if args.workload == "add_rmsnorm_quant":
+        return run_reference_norm(args, world)
     calls = workload_calls(args.workload)
     wcache = {}
 
@@ -868,6 +967,36 @@ def run_reference(args):
             "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": cores, **_host(), "kind": "oracle",
                              "sample": f"one call per step, cycling through the {args.workload} calls; M > 64 timed "
                                        "on 64 rows and scaled"},
+            "e2e": {"value": round(us, 1), "unit": "µs/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_reference_norm(args, world):
+    """The oracle's fused residual add + RMSNorm + quantisation, one call per step (M > 64
+    timed on 64 rows and scaled by M / 64: the step is row-separable)."""
+    from oracle import norm as onorm
+    calls = [(M, K) for K in inputs.NORM_KS for M in inputs.NORM_MS]
+
+    def one(c):
+        M, K = calls[c % len(calls)]
+        m = min(M, 64)
+        x = inputs.activation_bf16(m, K, 300 + c % len(calls)).float().numpy()
+        r = inputs.activation_bf16(m, K, 400 + c % len(calls)).float().numpy()
+        g = np.ones(K)
+        t0 = time.perf_counter()
+        onorm.add_rmsnorm_quant(x, r, g, 1e-6)
+        return (time.perf_counter() - t0) * M / m
+
+    for s in range(args.warmup):
+        one(s)
+    us = float(np.mean([one(args.warmup + s) for s in range(args.steps)])) * 1e6
+    line = {"impl": "reference", "metric": NORM_METRIC, "value": round(us, 1), "unit": "µs/call", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1000.0, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "add_rmsnorm_quant", "description": inputs.WORKLOADS["add_rmsnorm_quant"]},
+            "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": _threads(), **_host(), "kind": "oracle",
+                             "sample": "one call per step, cycling through the calls; M > 64 timed on 64 rows and "
+                                       "scaled"},
             "e2e": {"value": round(us, 1), "unit": "µs/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -915,6 +1044,8 @@ def run_gpu(args):
         if args.workload in BF16_WORKLOADS and not args.shape:
             line = measure_bf16(args, world, rank, dev, args.steps, args.warmup, args.detail, args.e2e_steps,
                                 args.cpu_baseline, args.workload)
+        elif args.workload == "add_rmsnorm_quant":
+            line = measure_norm(args, world, rank, dev, args.steps, args.warmup)
         else:
             line = measure_a8w8(args, world, rank, dev, args.workload, args.shape, args.steps, args.warmup,
                                 args.detail, args.e2e_steps, args.cpu_baseline)
@@ -931,6 +1062,8 @@ def run_gpu(args):
                 subs[w] = measure_bf16(args, world, rank, dev, min(args.steps, BF16_SUB_STEPS), 3, w == "lm_head", 0,
                                        False, w)
                 torch.cuda.empty_cache()
+            subs["add_rmsnorm_quant"] = measure_norm(args, world, rank, dev, min(args.steps, 20), 3)
+            torch.cuda.empty_cache()
             if rank == 0:
                 line["workloads"] = {w: compact(v) for w, v in subs.items()}
         if rank == 0:

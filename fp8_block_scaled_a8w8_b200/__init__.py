@@ -21,7 +21,7 @@ __all__ = [
     "gemm_bf16", "workspace_bytes", "Workspace", "dispatch_lookup", "dispatch_set_row", "dispatch_reset_table",
     "dispatch_list_configs", "dispatch_stats", "dispatch_reset_stats", "dispatch_dump_json", "dispatch_table_hash",
     "get_device_status", "status_string", "version", "OP_A8W8_BLOCKSCALE", "OP_BF16", "LIB_PATH",
-    "FLAG_STATIC_WEIGHTS", "gemm_a8w8_blockscale_noalloc", "test_set_wait_fault",
+    "FLAG_STATIC_WEIGHTS", "gemm_a8w8_blockscale_noalloc", "test_set_wait_fault", "add_rmsnorm_quant",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bs.so")
@@ -44,6 +44,8 @@ _c_void_p, _i64, _int, _sz, _u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 _PROTOS = {
     "fp8bs_quant_act_per_token_group": (_int, [_c_void_p, _i64, _i64, _i64, _c_void_p, _c_void_p, _int, _c_void_p]),
     "fp8bs_quant_weight_block128": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
+    "fp8bs_add_rmsnorm_quant": (_int, [_c_void_p, _c_void_p, _c_void_p, ctypes.c_float, _i64, _i64, _c_void_p,
+                                       _c_void_p, _c_void_p, _c_void_p]),
     "fp8bs_gemm_a8w8_blockscale": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
                                           _c_void_p, _sz, _c_void_p]),
     "fp8bs_gemm_a8w8_blockscale_ex": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
@@ -131,6 +133,30 @@ def quant_act_per_token_group(x: torch.Tensor, q: torch.Tensor | None = None, sc
            lib().fp8bs_quant_act_per_token_group(_ptr(x), M, K, x.stride(0), _ptr(q), _ptr(scale), group,
                                                  _stream(stream)))
     return q, scale
+
+
+def add_rmsnorm_quant(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6,
+                      residual_out: torch.Tensor | None = None, q: torch.Tensor | None = None,
+                      scale: torch.Tensor | None = None, stream=None):
+    """Fused residual add + RMSNorm + per-token 1x128 quantisation (fp8bs_add_rmsnorm_quant).
+    x, residual: bf16 [M, K] contiguous; gamma: bf16 [K]. Returns (residual_out bf16 [M, K],
+    codes float8_e4m3fn [M, K], scale float32 [M, K/128]); residual_out may be residual."""
+    for t in (x, residual, gamma):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("x, residual and gamma must be contiguous bf16 tensors")
+    M, K = x.shape
+    if residual.shape != (M, K) or gamma.shape != (K,):
+        raise ValueError("residual must be [M, K] and gamma [K]")
+    if residual_out is None:
+        residual_out = torch.empty_like(x)
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    if scale is None:
+        scale = torch.empty((M, K // 128), dtype=torch.float32, device=x.device)
+    _check("fp8bs_add_rmsnorm_quant",
+           lib().fp8bs_add_rmsnorm_quant(_ptr(x), _ptr(residual), _ptr(gamma), float(eps), M, K, _ptr(residual_out),
+                                         _ptr(q), _ptr(scale), _stream(stream)))
+    return residual_out, q, scale
 
 
 def quant_weight_block128(w: torch.Tensor, q: torch.Tensor | None = None, scale: torch.Tensor | None = None,

@@ -113,6 +113,23 @@ FP8BS_API fp8bs_status fp8bs_quant_act_per_token_group(const void* x_bf16, int64
   return from_cuda(launch_quant_act(x_bf16, M, K, ld_x, q_e4m3, a_scale, stream));
 }
 
+FP8BS_API fp8bs_status fp8bs_add_rmsnorm_quant(const void* x_bf16, const void* residual_bf16,
+                                                const void* gamma_bf16, float eps, int64_t M, int64_t K,
+                                                void* residual_out_bf16, void* q_e4m3, float* a_scale,
+                                                fp8bs_stream_t stream) {
+  if (!x_bf16 || !residual_bf16 || !gamma_bf16 || !residual_out_bf16 || !q_e4m3 || !a_scale || M <= 0 || K <= 0 ||
+      K % 128 != 0 || !(eps >= 0.f))
+    return FP8BS_ERR_INVALID_ARG;
+  if (M >= (int64_t(1) << 31) / (K / 128) || K > 32768) return FP8BS_ERR_UNSUPPORTED;
+  if (!aligned16(x_bf16) || !aligned16(residual_bf16) || !aligned16(gamma_bf16) || !aligned16(residual_out_bf16) ||
+      !aligned16(q_e4m3) || !aligned16(a_scale))
+    return FP8BS_ERR_ALIGNMENT;
+  fp8bs_status st = check_device();
+  if (st != FP8BS_OK) return st;
+  return from_cuda(
+      launch_add_rmsnorm_quant(x_bf16, residual_bf16, gamma_bf16, eps, residual_out_bf16, q_e4m3, a_scale, M, K, stream));
+}
+
 FP8BS_API fp8bs_status fp8bs_quant_weight_block128(const float* w_f32, int64_t N, int64_t K, void* q_e4m3,
                                                    float* w_scale, fp8bs_stream_t stream) {
   if (!w_f32 || !q_e4m3 || !w_scale || N <= 0 || K <= 0 || K % 128 != 0) return FP8BS_ERR_INVALID_ARG;

@@ -67,6 +67,8 @@ int set_max_dynamic_smem(const void* kernel, int bytes);
 // ---- launchers (return a cudaError_t value as int; 0 = success) ----
 int launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q, float* scale, void* stream);
 int launch_quant_weight(const float* w, int64_t N, int64_t K, void* q, float* scale, void* stream);
+int launch_add_rmsnorm_quant(const void* x, const void* residual, const void* gamma, float eps, void* residual_out,
+                             void* q, float* scale, int64_t M, int64_t K, void* stream);
 
 size_t gemv_workspace_bytes(int op, int64_t M, int64_t N, int64_t K, const KernelConfig& cfg);
 int launch_gemv_a8w8(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W,

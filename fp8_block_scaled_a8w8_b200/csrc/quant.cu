@@ -102,6 +102,116 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const float* __restri
   for (int i = 0; i < 4; ++i) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
 }
 
+// Fused residual add + RMSNorm + activation quantisation (the add_rmsnorm_quant step of
+// [mi210 docs/43] "43-ck-int8-gemm-gfx90a.md", Rounds 40-41, which feeds the GEMM), one
+// CTA per token row:
+//   h = bf16(float(x) + float(residual))          -> residual_out (may alias residual)
+//   r = 1 / sqrt(sum(h^2) / K + eps)              (float32; IEEE sqrt and division)
+//   y = (h * r) * gamma                           (float32)
+//   q, a_scale = the 1x128 activation quantiser of y (as quant_act_kernel)
+// Thread t holds the 16-byte vectors t, t + T, ... (T threads, at most kNormVpt vectors
+// each), so every load of the row is in flight at once and a half-warp covers one
+// 128-wide group; the sum of squares is reduced by warp shuffles and across warps in
+// shared memory. y stays in registers and is quantised straight from float32.
+constexpr int kNormVpt = 4;
+
+template <int VPT>
+__global__ void __launch_bounds__(1024) add_rmsnorm_quant_kernel(const uint16_t* x, const uint16_t* res,
+                                                                 const uint16_t* __restrict__ gamma, float eps,
+                                                                 uint16_t* res_out, uint8_t* __restrict__ q,
+                                                                 float* __restrict__ scale, int64_t M, int64_t K) {
+  __shared__ float warp_ss[32];
+  __shared__ float s_rinv;
+  pdl_trigger();
+  pdl_wait();
+  const int64_t row = blockIdx.x;
+  const int T = blockDim.x, t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const int64_t nv = K / 8;
+  const int64_t base = row * K;
+  float f[VPT][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int64_t v = t + int64_t(j) * T;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[j][i] = 0.f;
+    if (v < nv) {
+      // plain loads: residual and residual_out may be the same buffer
+      const uint4 xa = *reinterpret_cast<const uint4*>(x + base + 8 * v);
+      const uint4 ra = *reinterpret_cast<const uint4*>(res + base + 8 * v);
+      const uint32_t xw[4] = {xa.x, xa.y, xa.z, xa.w}, rw[4] = {ra.x, ra.y, ra.z, ra.w};
+      uint32_t hw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(__fadd_rn(bf16_lo(xw[i]), bf16_lo(rw[i])),
+                                                        __fadd_rn(bf16_hi(xw[i]), bf16_hi(rw[i])));
+        hw[i] = *reinterpret_cast<const uint32_t*>(&h2);
+        f[j][2 * i] = bf16_lo(hw[i]);
+        f[j][2 * i + 1] = bf16_hi(hw[i]);
+        ss = __fmaf_rn(f[j][2 * i], f[j][2 * i], ss);
+        ss = __fmaf_rn(f[j][2 * i + 1], f[j][2 * i + 1], ss);
+      }
+      *reinterpret_cast<uint4*>(res_out + base + 8 * v) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) ss = __fadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, off));
+  if (lane == 0) warp_ss[w] = ss;
+  __syncthreads();
+  if (t == 0) {
+    float tot = 0.f;
+    for (int i = 0; i < (T >> 5); ++i) tot = __fadd_rn(tot, warp_ss[i]);  // in warp order
+    s_rinv = __fdiv_rn(1.f, __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, float(K)), eps)));
+  }
+  __syncthreads();
+  const float rinv = s_rinv;
+  const int64_t G = K / 128;
+#pragma unroll
+  for (int j = 0; j < VPT; ++j) {
+    const int64_t v = t + int64_t(j) * T;
+    const bool valid = v < nv;
+    if (valid) {
+      const uint4 ga = ld_nc_v4(gamma + 8 * v);
+      const uint32_t gw[4] = {ga.x, ga.y, ga.z, ga.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        f[j][2 * i] = __fmul_rn(__fmul_rn(f[j][2 * i], rinv), bf16_lo(gw[i]));
+        f[j][2 * i + 1] = __fmul_rn(__fmul_rn(f[j][2 * i + 1], rinv), bf16_hi(gw[i]));
+      }
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[j][i]));
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float s = __fdiv_rn(amax, 448.f);
+    if (valid) {
+      uint2 out;
+      out.x = cvt4_e4m3(quant_div(f[j][0], s), quant_div(f[j][1], s), quant_div(f[j][2], s), quant_div(f[j][3], s));
+      out.y = cvt4_e4m3(quant_div(f[j][4], s), quant_div(f[j][5], s), quant_div(f[j][6], s), quant_div(f[j][7], s));
+      *reinterpret_cast<uint2*>(q + base + 8 * v) = out;
+      if ((lane & 15) == 0) scale[row * G + v / 16] = s;
+    }
+  }
+}
+
+int launch_add_rmsnorm_quant(const void* x, const void* residual, const void* gamma, float eps, void* residual_out,
+                             void* q, float* scale, int64_t M, int64_t K, void* stream) {
+  const int64_t nv = K / 8;
+  const int64_t per = (nv + 1023) / 1024;  // vectors per thread at 1024 threads
+  if (per > kNormVpt || M > 0x7FFFFFFF) return int(cudaErrorInvalidValue);
+  const int vpt = per <= 1 ? 1 : per <= 2 ? 2 : 4;
+  const int threads = int(((nv + vpt - 1) / vpt + 31) / 32 * 32);
+  auto args = [&](auto kernel) {
+    return launch_kernel(kernel, dim3(unsigned(M)), dim3(threads), 0, stream, static_cast<const uint16_t*>(x),
+                         static_cast<const uint16_t*>(residual), static_cast<const uint16_t*>(gamma), eps,
+                         static_cast<uint16_t*>(residual_out), static_cast<uint8_t*>(q), scale, M, K);
+  };
+  if (vpt == 1) return args(add_rmsnorm_quant_kernel<1>);
+  if (vpt == 2) return args(add_rmsnorm_quant_kernel<2>);
+  return args(add_rmsnorm_quant_kernel<4>);
+}
+
 int launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q, float* scale, void* stream) {
   const int64_t groups = M * (K / 128);
   const int64_t need = (groups + 15) / 16;  // 16 groups per 256-thread block per pass

@@ -34,6 +34,9 @@ LADDER_NK = (5120, 6144)
 # small-N bf16 GEMMs: (N, K, fp32 output?)
 BF16_NK = [(256, 6144, False), (32, 6144, False), (384, 5120, False), (1024, 5120, True), (128, 512, False)]
 BF16_MS = [1, 32, 576, 4096, 16384]
+# the fused residual add + RMSNorm + quantisation step feeding the decode / prefill GEMMs
+NORM_KS = [5120, 6144]
+NORM_MS = [1, 16, 2048, 8192]
 # the target lm_head of [aiter#7247] "Technical Details" / microbenchmark table (bf16 out)
 LM_HEAD_NK = (32320, 5120)
 LM_HEAD_MS = [24, 384, 1536, 2304, 3072]
@@ -47,6 +50,8 @@ WORKLOADS = {
     "ladder": "a8w8 blockscale dense M ladder, 512 M drawn from 1..8192 on (N,K)=(5120,6144)",
     "bf16_small_n": "bf16 x bf16 small-N GEMMs, M in {1,32,576,4096,16384} x (N,K) in "
                     "{(256,6144),(32,6144),(384,5120),(1024,5120) fp32 out,(128,512)}",
+    "add_rmsnorm_quant": "fused residual add + RMSNorm + 1x128 fp8 quantisation, M in {1,16,2048,8192} x "
+                         "K in {5120,6144}",
     "lm_head": "bf16 x bf16 large-N lm_head GEMM, M in {24,384,1536,2304,3072} on (N,K)=(32320,5120), bf16 out",
 }
 

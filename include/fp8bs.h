@@ -84,6 +84,27 @@ fp8bs_status fp8bs_quant_act_per_token_group(const void* x_bf16, int64_t M, int6
                                              fp8bs_stream_t stream);
 
 /*
+ * Fused residual add + RMSNorm + activation quantisation: the step that produces the
+ * a8w8 GEMM's input (add_rmsnorm_quant in the decode kernel table of [mi210 docs/43]
+ * "43-ck-int8-gemm-gfx90a.md", Rounds 40-41). For every token row m:
+ *   h[m,k]  = bf16(float(x[m,k]) + float(residual[m,k]))   written to residual_out
+ *   r[m]    = 1 / sqrt(sum_k h[m,k]^2 / K + eps)             float32
+ *   y[m,k]  = (h[m,k] * r[m]) * gamma[k]                     float32, never rounded to bf16
+ *   q, a_scale = the per-token 1x128 quantisation of y (as fp8bs_quant_act_per_token_group)
+ * x_bf16, residual_bf16: device, bf16 [M, K]; gamma_bf16: device, bf16 [K];
+ * residual_out_bf16: device, bf16 [M, K], written (it may be residual_bf16 itself);
+ * q_e4m3: device, e4m3 [M, K], written; a_scale: device, float32 [M, K/128], written.
+ * Requires K % 128 == 0, eps >= 0 (FP8BS_ERR_INVALID_ARG otherwise) and K <= 32768
+ * (FP8BS_ERR_UNSUPPORTED otherwise: one CTA holds a row in registers). residual_out is
+ * bit-identical to the oracle's; the mean square is a float32 sum, so a code may differ
+ * from the float64 oracle's by one step where y / a_scale is within float32 error of a
+ * rounding midpoint.
+ */
+fp8bs_status fp8bs_add_rmsnorm_quant(const void* x_bf16, const void* residual_bf16, const void* gamma_bf16,
+                                     float eps, int64_t M, int64_t K, void* residual_out_bf16, void* q_e4m3,
+                                     float* a_scale, fp8bs_stream_t stream);
+
+/*
  * Weight quantisation, per 128x128 block ([cookbook#8]: weight_block_size [128,128]).
  * For every block (nb, g): amax over rows 128nb .. min(N,128nb+128)-1 and columns
  * 128g .. 128g+127; w_scale[nb,g] = amax / 448; codes as for activations.
