@@ -36,6 +36,7 @@ Modules:
   gemm      -- a8w8 block-scaled GEMM and plain bf16 GEMM in float64
   metrics   -- relative L2, error ratio, bf16 ulp
   norm      -- fused residual add + RMSNorm + activation quantisation
+  mx        -- MX32 variant: E8M0 scales, 1x32 activation groups, 32x32 weight blocks
   dispatch  -- the padded-M lookup walk and the census deduplication rule
 
 Parity status of every function is listed in each module's header; every
@@ -43,4 +44,4 @@ function here is pinned by a ``-m "not gpu"`` test in ``tests/test_oracle_*.py``
 against something other than itself.
 """
 
-from . import e4m3, bf16, quant, gemm, metrics, dispatch, norm  # noqa: F401
+from . import e4m3, bf16, quant, gemm, metrics, dispatch, norm, mx  # noqa: F401
