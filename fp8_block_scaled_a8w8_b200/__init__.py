@@ -22,6 +22,7 @@ __all__ = [
     "dispatch_list_configs", "dispatch_stats", "dispatch_reset_stats", "dispatch_dump_json", "dispatch_table_hash",
     "get_device_status", "status_string", "version", "OP_A8W8_BLOCKSCALE", "OP_BF16", "LIB_PATH",
     "FLAG_STATIC_WEIGHTS", "gemm_a8w8_blockscale_noalloc", "test_set_wait_fault", "add_rmsnorm_quant",
+    "quant_act_mx32", "quant_weight_mx32", "gemm_a8w8_mx32", "mx32_workspace_bytes",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8bs.so")
@@ -44,6 +45,11 @@ _c_void_p, _i64, _int, _sz, _u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
 _PROTOS = {
     "fp8bs_quant_act_per_token_group": (_int, [_c_void_p, _i64, _i64, _i64, _c_void_p, _c_void_p, _int, _c_void_p]),
     "fp8bs_quant_weight_block128": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
+    "fp8bs_quant_act_mx32": (_int, [_c_void_p, _i64, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
+    "fp8bs_quant_weight_mx32": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p, _c_void_p]),
+    "fp8bs_mx32_workspace_bytes": (_sz, [_i64, _i64, _i64, _i64]),
+    "fp8bs_gemm_a8w8_mx32": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64, _i64,
+                                    _c_void_p, _sz, _c_void_p]),
     "fp8bs_add_rmsnorm_quant": (_int, [_c_void_p, _c_void_p, _c_void_p, ctypes.c_float, _i64, _i64, _c_void_p,
                                        _c_void_p, _c_void_p, _c_void_p]),
     "fp8bs_gemm_a8w8_blockscale": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
@@ -157,6 +163,65 @@ def add_rmsnorm_quant(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tens
            lib().fp8bs_add_rmsnorm_quant(_ptr(x), _ptr(residual), _ptr(gamma), float(eps), M, K, _ptr(residual_out),
                                          _ptr(q), _ptr(scale), _stream(stream)))
     return residual_out, q, scale
+
+
+def quant_act_mx32(x: torch.Tensor, q: torch.Tensor | None = None, e8m0: torch.Tensor | None = None, stream=None):
+    """MX32 activation quantisation (fp8bs_quant_act_mx32): x bf16 [M, K] (unit stride along K).
+    Returns (codes float8_e4m3fn [M, K], E8M0 exponents uint8 [M, K/32])."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D bf16 tensor with unit stride along K")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    if e8m0 is None:
+        e8m0 = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
+    _check("fp8bs_quant_act_mx32",
+           lib().fp8bs_quant_act_mx32(_ptr(x), M, K, x.stride(0), _ptr(q), _ptr(e8m0), _stream(stream)))
+    return q, e8m0
+
+
+def quant_weight_mx32(w: torch.Tensor, q: torch.Tensor | None = None, e8m0: torch.Tensor | None = None,
+                      stream=None):
+    """MX32 weight quantisation (32x32 blocks): w float32 [N, K] contiguous. Returns (codes
+    float8_e4m3fn [N, K], E8M0 exponents uint8 [ceil(N/32), K/32])."""
+    if w.dtype != torch.float32 or w.dim() != 2 or not w.is_contiguous():
+        raise ValueError("w must be a contiguous 2-D float32 tensor")
+    N, K = w.shape
+    if q is None:
+        q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
+    if e8m0 is None:
+        e8m0 = torch.empty(((N + 31) // 32, K // 32), dtype=torch.uint8, device=w.device)
+    _check("fp8bs_quant_weight_mx32", lib().fp8bs_quant_weight_mx32(_ptr(w), N, K, _ptr(q), _ptr(e8m0), _stream(stream)))
+    return q, e8m0
+
+
+def mx32_workspace_bytes(batch: int, M: int, N: int, K: int) -> int:
+    return int(lib().fp8bs_mx32_workspace_bytes(batch, M, N, K))
+
+
+def gemm_a8w8_mx32(A: torch.Tensor, a_e8m0: torch.Tensor, W: torch.Tensor, w_e8m0: torch.Tensor,
+                   out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """MX32 GEMM (fp8bs_gemm_a8w8_mx32). 2-D operands (A [M, K], W [N, K]) are one GEMM;
+    3-D stacks (A [b, M, K], W [b, N, K]) are b independent GEMMs. Returns out bf16 [.., M, N]."""
+    if not (_is_byte(A) and _is_byte(W)) or A.dim() != W.dim() or A.dim() not in (2, 3):
+        raise ValueError("A and W must be 2-D or 3-D one-byte (e4m3 code) tensors of the same rank")
+    batch = A.shape[0] if A.dim() == 3 else 1
+    M, K = A.shape[-2:]
+    N = W.shape[-2]
+    for t in (A, a_e8m0, W, w_e8m0):
+        if not t.is_contiguous():
+            raise ValueError("operands must be contiguous")
+    if out is None:
+        out = torch.empty(((batch,) if A.dim() == 3 else ()) + (M, N), dtype=torch.bfloat16, device=A.device)
+    need = mx32_workspace_bytes(batch, M, N, K)
+    if workspace is None:
+        workspace = _workspace_for(A.device, need)
+    ws_ptr = _ptr(workspace) if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("fp8bs_gemm_a8w8_mx32",
+           lib().fp8bs_gemm_a8w8_mx32(_ptr(A), _ptr(a_e8m0), _ptr(W), _ptr(w_e8m0), _ptr(out), batch, M, N, K, ws_ptr,
+                                      ws_len, _stream(stream)))
+    return out
 
 
 def quant_weight_block128(w: torch.Tensor, q: torch.Tensor | None = None, scale: torch.Tensor | None = None,

@@ -130,6 +130,31 @@ FP8BS_API fp8bs_status fp8bs_add_rmsnorm_quant(const void* x_bf16, const void* r
       launch_add_rmsnorm_quant(x_bf16, residual_bf16, gamma_bf16, eps, residual_out_bf16, q_e4m3, a_scale, M, K, stream));
 }
 
+FP8BS_API fp8bs_status fp8bs_quant_act_mx32(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, void* q_e4m3,
+                                             uint8_t* a_e8m0, fp8bs_stream_t stream) {
+  if (!x_bf16 || !q_e4m3 || !a_e8m0 || M <= 0 || K <= 0 || K % 32 != 0 || ld_x < K) return FP8BS_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 31) / (K / 32)) return FP8BS_ERR_UNSUPPORTED;
+  if (!aligned16(x_bf16) || !aligned16(q_e4m3) || ld_x % 8 != 0) return FP8BS_ERR_ALIGNMENT;
+  fp8bs_status st = check_device();
+  if (st != FP8BS_OK) return st;
+  return from_cuda(launch_quant_act_mx32(x_bf16, M, K, ld_x, q_e4m3, a_e8m0, stream));
+}
+
+FP8BS_API fp8bs_status fp8bs_quant_weight_mx32(const float* w_f32, int64_t N, int64_t K, void* q_e4m3,
+                                               uint8_t* w_e8m0, fp8bs_stream_t stream) {
+  if (!w_f32 || !q_e4m3 || !w_e8m0 || N <= 0 || K <= 0 || K % 32 != 0) return FP8BS_ERR_INVALID_ARG;
+  if (((N + 31) / 32) * (K / 32) > (int64_t(1) << 31) / 32) return FP8BS_ERR_UNSUPPORTED;
+  if (!aligned16(w_f32) || !aligned16(q_e4m3)) return FP8BS_ERR_ALIGNMENT;
+  fp8bs_status st = check_device();
+  if (st != FP8BS_OK) return st;
+  return from_cuda(launch_quant_weight_mx32(w_f32, N, K, q_e4m3, w_e8m0, stream));
+}
+
+FP8BS_API size_t fp8bs_mx32_workspace_bytes(int64_t batch, int64_t M, int64_t N, int64_t K) {
+  if (batch <= 0 || M <= 0 || N <= 0 || K <= 0 || K % 128 != 0) return 0;
+  return mx_workspace_bytes(batch, M, N, K);
+}
+
 FP8BS_API fp8bs_status fp8bs_quant_weight_block128(const float* w_f32, int64_t N, int64_t K, void* q_e4m3,
                                                    float* w_scale, fp8bs_stream_t stream) {
   if (!w_f32 || !q_e4m3 || !w_scale || N <= 0 || K <= 0 || K % 128 != 0) return FP8BS_ERR_INVALID_ARG;
@@ -241,12 +266,32 @@ FP8BS_API fp8bs_status fp8bs_gemm_bf16(const void* A_bf16, const void* W_bf16, v
   return from_cuda(e);
 }
 
+FP8BS_API fp8bs_status fp8bs_gemm_a8w8_mx32(const void* A_e4m3, const uint8_t* a_e8m0, const void* W_e4m3,
+                                            const uint8_t* w_e8m0, void* out_bf16, int64_t batch, int64_t M,
+                                            int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                                            fp8bs_stream_t stream) {
+  if (!A_e4m3 || !a_e8m0 || !W_e4m3 || !w_e8m0 || !out_bf16 || batch <= 0) return FP8BS_ERR_INVALID_ARG;
+  fp8bs_status st = check_gemm_shape(M, N, K, 128);
+  if (st != FP8BS_OK) return st;
+  if (batch > 65535 || batch * M >= (int64_t(1) << 31) / (K / 32) || batch * ((N + 31) / 32) * (K / 32) >= (int64_t(1) << 31))
+    return FP8BS_ERR_UNSUPPORTED;
+  if (!aligned16(A_e4m3) || !aligned16(W_e4m3) || !aligned16(out_bf16) || !aligned16(a_e8m0) || !aligned16(w_e8m0))
+    return FP8BS_ERR_ALIGNMENT;
+  st = check_device();
+  if (st != FP8BS_OK) return st;
+  const size_t need = mx_workspace_bytes(batch, M, N, K);
+  if (need && (!workspace || workspace_bytes < need)) return FP8BS_ERR_WORKSPACE;
+  if (need && !aligned16(workspace)) return FP8BS_ERR_ALIGNMENT;
+  return from_cuda(launch_gemm_mx32(A_e4m3, a_e8m0, W_e4m3, w_e8m0, out_bf16, batch, M, N, K, workspace, stream,
+                                    unsigned(kWaitLimitNs)));
+}
+
 FP8BS_API fp8bs_status fp8bs_get_device_status(fp8bs_stream_t stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP8BS_ERR_CUDA;
   const unsigned int a = take_status_tc(), b = take_status_gemv_tma(), c = take_status_gemv_umma(),
-                     d = take_status_fp8();
-  if (a == ~0u || b == ~0u || c == ~0u || d == ~0u) return FP8BS_ERR_CUDA;
-  const unsigned int v = a | b | c | d;
+                     d = take_status_fp8(), e = take_status_mx();
+  if (a == ~0u || b == ~0u || c == ~0u || d == ~0u || e == ~0u) return FP8BS_ERR_CUDA;
+  const unsigned int v = a | b | c | d | e;
   return (v & kStatusTimeout) ? FP8BS_ERR_TIMEOUT : FP8BS_OK;
 }
 

@@ -1,0 +1,502 @@
+// MX32 variant of the a8w8 GEMM on the tensor core's own block scaling: tcgen05.mma
+// kind::mxf8f6f4.block_scale with E8M0 scale factors in TMEM.
+//
+//   out[b,m,n] = sum_g 2^(ea[b,m,g] + ew[b,n/32,g] - 254) * sum_{k in g} A[b,m,k] W[b,n,k]
+//
+// with 32-wide K groups g, 1x32 activation scales and 32x32 weight-block scales
+// ([aiter#7247] "Motivation": MX32, w_scale_block 32x32; "Technical Details": the dense
+// shapes and the batched b = 8, N = 1024, K = 4096 GEMM). Because the scales are powers of
+// two the hardware applies them inside the MMA, so the fp32 accumulator stays in TMEM
+// over the whole K range -- no per-group promotion by the epilogue, unlike the fp32-scale
+// 128-block kernels.
+//
+// Tiles of 128 rows x 192 columns, persistent CTAs, K staged 128 at a time (four K = 32
+// MMAs, each selecting its scale byte with the instruction's scale-factor ids).
+//   warp 0        TMA producer: A box 128 rows x 128 bytes, W box 192 rows x 128 bytes
+//   warp 1        TMEM allocator and MMA issuer
+//   warps 4..7    scale-factor writers: per stage, tcgen05.st of the tile's scale bytes
+//                 into a TMEM slot -- row m at lane m % 32 of every 32-lane subpartition,
+//                 column m / 32, one byte per K group (measured layout of the block-scaled
+//                 MMA's scale-factor operands)
+//   warps 8..15   epilogue: TMEM -> bf16 -> shared memory -> TMA store (two TMEM
+//                 accumulators alternate between tiles)
+// Small tile counts split K: each split stores the rows < M of its fp32 tile, the last to
+// arrive (gpu-scope acq_rel counter) sums them in split order and writes bf16.
+// Every wait is bounded; on expiry the CTA raises its abort flag and the status word,
+// drains what it issued and frees TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace fp8bs {
+
+FP8BS_DEFINE_STATUS(mx)
+
+constexpr int kMxThreads = 512;
+constexpr int kMxBM = 128, kMxBN = 192;
+constexpr int kMxStages = 4;
+constexpr int kMxABytes = kMxBM * 128, kMxBBytes = kMxBN * 128, kMxStageBytes = kMxABytes + kMxBBytes;
+constexpr int kMxEpiWarps = 8;
+constexpr int kMxOutBytes = kMxEpiWarps * 2048;  // one 32 x 32 bf16 staging box per epilogue warp
+constexpr size_t kMxSmemBytes = size_t(kMxStages) * kMxStageBytes + kMxOutBytes + 1024 + 256;
+constexpr uint32_t kMxSfBase = 2 * kMxBN;  // TMEM: [2 accumulators][scale-factor slots of 32 columns]
+static_assert(kMxSfBase + 32 * kMxStages <= 512, "TMEM budget");
+static_assert(kMxStageBytes % 1024 == 0, "stage alignment");
+static_assert(kMxSmemBytes <= 232448, "shared memory per block");
+
+struct MxParams {
+  const uint8_t* a_e;   // [batch][M][K/32] E8M0
+  const uint8_t* w_e;   // [batch][ceil(N/32)][K/32] E8M0
+  __nv_bfloat16* out;   // [batch][M][N]
+  int M, N, K32, KB, NB32, batch;
+  int m_tiles, n_tiles, splits;
+  float* part;          // splits > 1: [items][kMxBM][kMxBN] float32 partial tiles
+  unsigned* counter;    // splits > 1: [tiles]
+  uint32_t wait_ns;
+};
+
+// Block-scaled instruction descriptor: E4M3 x E4M3, both K-major, E8M0 scale factors
+// (bit 23), B scale-factor id at bits 4-5, A's at bits 29-30, N >> 3 at 17-22, M >> 4 at 24-28.
+__host__ __device__ constexpr uint32_t mx_idesc(uint32_t m, uint32_t n, uint32_t sf_id) {
+  return (sf_id << 4) | ((n >> 3) << 17) | (1u << 23) | ((m >> 4) << 24) | (sf_id << 29);
+}
+
+__device__ __forceinline__ void mx_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mx_tmem_st_x4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void mx_tmem_st_x8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+__device__ __forceinline__ void mx_tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void mx_tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                               int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t mx_timer() {
+  uint32_t t;
+  asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
+  return t;
+}
+// Bounded wait (sleeping in try_wait between checks of the abort flag and the clock).
+__device__ __forceinline__ bool mx_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t t0 = mx_timer();
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(50000u)
+        : "memory");
+    if (ok) return true;
+    if (*abort) return false;
+    if (mx_timer() - t0 > limit) {
+      *abort = 1;
+      atomicOr(&g_status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void mx_drain(uint32_t bar, uint32_t parity, uint32_t limit) {
+  const uint32_t t0 = mx_timer();
+  while (!mbar_try_wait(bar, parity))
+    if (mx_timer() - t0 > limit) {
+      atomicOr(&g_status, kStatusTimeout);
+      return;
+    }
+}
+
+__device__ __forceinline__ uint32_t mx_pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void mx_epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// item -> (split, tile); tile -> (tm fastest, tn, batch)
+struct MxItem {
+  int sp, tile, tm, tn, bt, kb0, kb1;
+};
+__device__ __forceinline__ MxItem mx_item(const MxParams& p, int item) {
+  MxItem r;
+  r.tile = item / p.splits;
+  r.sp = item - r.tile * p.splits;
+  r.tm = r.tile % p.m_tiles;
+  const int rest = r.tile / p.m_tiles;
+  r.tn = rest % p.n_tiles;
+  r.bt = rest / p.n_tiles;
+  r.kb0 = p.KB * r.sp / p.splits;
+  r.kb1 = p.KB * (r.sp + 1) / p.splits;
+  return r;
+}
+
+template <bool kSplitK>
+__global__ void __launch_bounds__(kMxThreads, 1)
+    gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmOut, const MxParams p) {
+  constexpr int S = kMxStages;
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* out_stage = smem + size_t(S) * kMxStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + kMxOutBytes);
+  // bars: full[S], empty[S], sf_full[S], tfull[2], tempty[2], drain
+  uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+  uint32_t* tmem_slot = misc;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  volatile unsigned* s_old = reinterpret_cast<volatile unsigned*>(misc + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + S + s); };
+  auto sf_full_bar = [&](int s) { return smem_u32(bars + 2 * S + s); };
+  auto tfull_bar = [&](int b) { return smem_u32(bars + 3 * S + b); };
+  auto tempty_bar = [&](int b) { return smem_u32(bars + 3 * S + 2 + b); };
+  const uint32_t drain_bar = smem_u32(bars + 3 * S + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+      mbar_init(sf_full_bar(s), 4);  // the four scale-factor writer warps
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), kMxEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_wait();
+  const uint32_t tmem_base = *tmem_slot;
+  const int splits = kSplitK ? p.splits : 1;
+  const int items = p.batch * p.m_tiles * p.n_tiles * splits;
+  const uint32_t lim = p.wait_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+        const MxItem w = mx_item(p, item);
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int s = it % S;
+          if (!mx_wait(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(smem + size_t(s) * kMxStageBytes);
+          mbar_arrive_expect_tx(full_bar(s), kMxStageBytes);
+          mx_tma_load_3d(dst, &tmA, full_bar(s), kb * 128, w.tm * kMxBM, w.bt);
+          mx_tma_load_3d(dst + kMxABytes, &tmB, full_bar(s), kb * 128, w.tn * kMxBN, w.bt);
+        }
+      }
+      for (int j = it > S ? it - S : 0; j < it; ++j) mx_drain(full_bar(j % S), (j / S) & 1, lim);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int it = 0, tile_it = 0;
+      bool ok = true, issued = false;
+      for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++tile_it) {
+        const MxItem w = mx_item(p, item);
+        const int b = tile_it & 1;
+        if (!mx_wait(tempty_bar(b), ((tile_it >> 1) & 1) ^ 1, abort_flag, lim)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + uint32_t(b * kMxBN);
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int s = it % S;
+          if (!mx_wait(full_bar(s), (it / S) & 1, abort_flag, lim) ||
+              !mx_wait(sf_full_bar(s), (it / S) & 1, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + size_t(s) * kMxStageBytes);
+          const uint64_t adesc = sw128_kmajor_desc(a_addr), bdesc = sw128_kmajor_desc(a_addr + kMxABytes);
+          const uint32_t sfa = tmem_base + kMxSfBase + uint32_t(32 * s), sfb = sfa + 16;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mx_mma(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, mx_idesc(kMxBM, kMxBN, kk), sfa, sfb,
+                   (kb > w.kb0 || kk > 0) ? 1u : 0u);
+          issued = true;
+          umma_commit(empty_bar(s));  // the stage and its scale-factor slot are free
+        }
+        if (ok) umma_commit(tfull_bar(b));
+      }
+      if (issued) {
+        umma_commit(drain_bar);
+        mx_drain(drain_bar, 0, lim);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ scale-factor writers
+    // warp q writes TMEM lanes 32q..32q+31 (every subpartition holds the same copy)
+    const uint32_t lane_addr = tmem_base + (uint32_t(32 * (warp & 3)) << 16);
+    int it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+      const MxItem w = mx_item(p, item);
+      const uint8_t* arow = p.a_e + (int64_t(w.bt) * p.M) * p.K32;
+      const uint8_t* wrow = p.w_e + (int64_t(w.bt) * p.NB32) * p.K32;
+      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+        const int s = it % S;
+        // scale bytes of the four K groups of this stage: 4 consecutive bytes per row / block
+        uint32_t sa[4], sb[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int r = w.tm * kMxBM + lane + 32 * j;
+          sa[j] = r < p.M ? __ldg(reinterpret_cast<const uint32_t*>(arow + int64_t(r) * p.K32 + 4 * kb)) : 0x7F7F7F7Fu;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int nb = w.tn * (kMxBN / 32) + j;
+          sb[j] = (j < kMxBN / 32 && nb < p.NB32)
+                      ? __ldg(reinterpret_cast<const uint32_t*>(wrow + int64_t(nb) * p.K32 + 4 * kb))
+                      : 0x7F7F7F7Fu;
+        }
+        if (!__all_sync(0xffffffffu, mx_wait(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, lim))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t slot = lane_addr + kMxSfBase + uint32_t(32 * s);
+        mx_tmem_st_x4(slot, sa[0], sa[1], sa[2], sa[3]);  // column j: rows 32j + lane
+        mx_tmem_st_x8(slot + 16, sb);                      // column j: output columns 32j .. 32j + 31
+        mx_tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_full_bar(s));
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ epilogue warps 8..15
+    const int e = warp - 8, q = warp & 3, h = e >> 2;  // lane quarter, 96-column half
+    const uint32_t lane_addr = tmem_base + (uint32_t(32 * q) << 16);
+    const uint32_t stage = smem_u32(out_stage + e * 2048);
+    int tile_it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < items && (kSplitK || ok); item += gridDim.x, ++tile_it) {
+      const MxItem w = mx_item(p, item);
+      const int b = tile_it & 1;
+      const int row0 = w.tm * kMxBM + 32 * q;
+      const int col_base = w.tn * kMxBN + h * (kMxBN / 2);
+      if (ok && !__all_sync(0xffffffffu, mx_wait(tfull_bar(b), (tile_it >> 1) & 1, abort_flag, lim))) ok = false;
+      if (ok) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < kMxBN / 64; ++c) {  // 3 chunks of 32 columns
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(lane_addr + uint32_t(b * kMxBN + h * (kMxBN / 2) + 32 * c), r);
+          tmem_ld_wait();
+          if (c == kMxBN / 64 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(b));
+          }
+          const int col0 = col_base + 32 * c;
+          if constexpr (!kSplitK) {
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t addr = stage + uint32_t(lane * 64 + 16 * (j ^ ((lane >> 1) & 3)));
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                           "r"(mx_pack_bf16x2(__uint_as_float(r[8 * j]), __uint_as_float(r[8 * j + 1]))),
+                           "r"(mx_pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]))),
+                           "r"(mx_pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]))),
+                           "r"(mx_pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7])))
+                           : "memory");
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+              asm volatile(
+                  "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                      reinterpret_cast<uint64_t>(&tmOut)),
+                  "r"(col0), "r"(row0), "r"(w.bt), "r"(stage)
+                  : "memory");
+              asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+          } else {
+            const int row = row0 + lane;
+            if (row < p.M) {
+              float* dst = p.part + (int64_t(item) * kMxBM + 32 * q + lane) * kMxBN + h * (kMxBN / 2) + 32 * c;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                __stcg(reinterpret_cast<float4*>(dst + j),
+                       make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                   __uint_as_float(r[j + 3])));
+            }
+          }
+        }
+      }
+      if constexpr (kSplitK) {
+        // publish this split; the last split of the tile sums the partials in split order
+        mx_epi_bar();
+        if (threadIdx.x == 256) *s_old = (!ok || *abort_flag) ? ~0u : atom_add_acq_rel_gpu(p.counter + w.tile, 1u);
+        mx_epi_bar();
+        if (*s_old == unsigned(p.splits - 1)) {
+          const int row = row0 + lane;
+          if (row < p.M) {
+#pragma unroll 1
+            for (int c = 0; c < kMxBN / 64; ++c) {
+              float sum[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sum[j] = 0.f;
+#pragma unroll 1
+              for (int sp = 0; sp < p.splits; ++sp) {
+                const float* src = p.part + ((int64_t(w.tile) * p.splits + sp) * kMxBM + 32 * q + lane) * kMxBN +
+                                   h * (kMxBN / 2) + 32 * c;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                  const float4 f = __ldcg(reinterpret_cast<const float4*>(src + j));
+                  sum[j] += f.x;
+                  sum[j + 1] += f.y;
+                  sum[j + 2] += f.z;
+                  sum[j + 3] += f.w;
+                }
+              }
+              const int col0 = col_base + 32 * c;
+              __nv_bfloat16* dst = p.out + (int64_t(w.bt) * p.M + row) * p.N + col0;
+#pragma unroll
+              for (int j = 0; j < 32; j += 8)
+                if (col0 + j < p.N)
+                  *reinterpret_cast<uint4*>(dst + j) =
+                      make_uint4(mx_pack_bf16x2(sum[j], sum[j + 1]), mx_pack_bf16x2(sum[j + 2], sum[j + 3]),
+                                 mx_pack_bf16x2(sum[j + 4], sum[j + 5]), mx_pack_bf16x2(sum[j + 6], sum[j + 7]));
+            }
+          }
+          if (threadIdx.x == 256) p.counter[w.tile] = 0u;
+        }
+      } else {
+        if (!ok) break;
+      }
+    }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+static bool make_map_3d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int esz, int64_t inner, int64_t rows,
+                        int64_t batch, int box_inner, int box_rows, CUtensorMapSwizzle sw) {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  if (!enc) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  cuuint64_t dims[3] = {cuuint64_t(inner), cuuint64_t(rows), cuuint64_t(batch)};
+  cuuint64_t strides[2] = {cuuint64_t(inner * esz), cuuint64_t(inner * rows * esz)};
+  cuuint32_t box[3] = {cuuint32_t(box_inner), cuuint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  std::memset(m, 0, sizeof(*m));
+  return enc(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int mx_splits(int64_t batch, int64_t M, int64_t N, int64_t K) {
+  const int64_t kb = K / 128;
+  const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + kMxBN - 1) / kMxBN);
+  const int64_t sms = device_sm_count();
+  int64_t sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({(sms + tiles - 1) / tiles, kb / 2, 16});
+  sp = std::max<int64_t>(1, std::min(sp, kb));
+  if (sp > 1 && tiles > kMaxCounters) sp = 1;
+  return int(sp);
+}
+
+size_t mx_workspace_bytes(int64_t batch, int64_t M, int64_t N, int64_t K) {
+  const int sp = mx_splits(batch, M, N, K);
+  if (sp == 1) return 0;
+  const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + kMxBN - 1) / kMxBN);
+  return kCounterBytes + size_t(tiles) * sp * kMxBM * kMxBN * sizeof(float);
+}
+
+int launch_gemm_mx32(const void* A, const uint8_t* a_e, const void* W, const uint8_t* w_e, void* out, int64_t batch,
+                     int64_t M, int64_t N, int64_t K, void* ws, void* stream, unsigned wait_ns) {
+  MxParams p{};
+  p.a_e = a_e;
+  p.w_e = w_e;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.M = int(M);
+  p.N = int(N);
+  p.K32 = int(K / 32);
+  p.KB = int(K / 128);
+  p.NB32 = int((N + 31) / 32);
+  p.batch = int(batch);
+  p.m_tiles = int((M + kMxBM - 1) / kMxBM);
+  p.n_tiles = int((N + kMxBN - 1) / kMxBN);
+  p.splits = mx_splits(batch, M, N, K);
+  p.wait_ns = wait_ns;
+  if (p.splits > 1) {
+    if (!ws) return int(cudaErrorInvalidValue);
+    p.counter = static_cast<unsigned*>(ws);
+    p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
+  }
+  CUtensorMap ma, mb, mo;
+  if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, batch, 128, kMxBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_3d(&mb, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, batch, 128, kMxBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_3d(&mo, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, batch, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return int(cudaErrorInvalidValue);
+  const int items = p.batch * p.m_tiles * p.n_tiles * p.splits;
+  const int grid = std::min(items, device_sm_count());
+  if (p.splits > 1) {
+    if (const int e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_mx_kernel<true>), int(kMxSmemBytes)))
+      return e;
+    return launch_kernel(gemm_mx_kernel<true>, dim3(grid), dim3(kMxThreads), kMxSmemBytes, stream, ma, mb, mo, p);
+  }
+  if (const int e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_mx_kernel<false>), int(kMxSmemBytes)))
+    return e;
+  return launch_kernel(gemm_mx_kernel<false>, dim3(grid), dim3(kMxThreads), kMxSmemBytes, stream, ma, mb, mo, p);
+}
+
+}  // namespace fp8bs

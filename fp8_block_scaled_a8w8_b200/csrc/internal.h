@@ -57,6 +57,7 @@ unsigned int take_status_tc();
 unsigned int take_status_gemv_tma();
 unsigned int take_status_gemv_umma();
 unsigned int take_status_fp8();
+unsigned int take_status_mx();
 
 // Device properties, cached per device.
 int device_sm_count();
@@ -67,6 +68,8 @@ int set_max_dynamic_smem(const void* kernel, int bytes);
 // ---- launchers (return a cudaError_t value as int; 0 = success) ----
 int launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q, float* scale, void* stream);
 int launch_quant_weight(const float* w, int64_t N, int64_t K, void* q, float* scale, void* stream);
+int launch_quant_act_mx32(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q, void* ecode, void* stream);
+int launch_quant_weight_mx32(const float* w, int64_t N, int64_t K, void* q, void* ecode, void* stream);
 int launch_add_rmsnorm_quant(const void* x, const void* residual, const void* gamma, float eps, void* residual_out,
                              void* q, float* scale, int64_t M, int64_t K, void* stream);
 
@@ -104,6 +107,11 @@ bool make_tma_2d_bf16_store(CUtensorMap* m, void* ptr, int64_t rows, int64_t col
 size_t fp8_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, const KernelConfig& cfg);
 int launch_fp8_tc(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W, const float* w_scale,
                   void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream);
+// MX32 GEMM (E8M0 scales on 32-wide K groups, hardware block scaling), batch >= 1.
+size_t mx_workspace_bytes(int64_t batch, int64_t M, int64_t N, int64_t K);
+int launch_gemm_mx32(const void* A, const uint8_t* a_e, const void* W, const uint8_t* w_e, void* out, int64_t batch,
+                     int64_t M, int64_t N, int64_t K, void* ws, void* stream, unsigned wait_ns);
+
 // CTA-pair kernel (no split K, no workspace) and the clusters of two that fit at once.
 int launch_fp8_pair(int halves, const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
                     int64_t M, int64_t N, int64_t K, void* stream);

@@ -5,6 +5,8 @@
 // cvt.rn.satfinite.e4m3x2.f32 -- so the codes and scales equal the CPU
 // oracle's bit for bit. A group whose amax is 0 gets scale 0 and codes +-0.
 // ([cookbook#8]: the checkpoint is block quantised, weight_block_size [128,128].)
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -210,6 +212,121 @@ int launch_add_rmsnorm_quant(const void* x, const void* residual, const void* ga
   if (vpt == 1) return args(add_rmsnorm_quant_kernel<1>);
   if (vpt == 2) return args(add_rmsnorm_quant_kernel<2>);
   return args(add_rmsnorm_quant_kernel<4>);
+}
+
+// ---------------------------------------------------------------- MX32 quantisers
+// MX32 variant ([aiter#7247] "Motivation": 32x32 weight scale blocks): E8M0 scales
+// (value 2^(code - 127)) on 1x32 activation groups and 32x32 weight blocks. The exponent
+// is the smallest that keeps the group within the e4m3 range, read exactly from the
+// bits of r = amax / 448 (one IEEE float32 division): e = ceil(log2 r); code = e + 127
+// clamped to [0, 254]; amax == 0 gives code 0. Codes are e4m3_rn_satfinite(x * 2^-e), an
+// exact power-of-two scaling (rounded once only where the product is float32-subnormal).
+__device__ __forceinline__ int mx_code_for_amax(float amax) {
+  if (amax == 0.f) return 0;
+  const uint32_t b = __float_as_uint(__fdiv_rn(amax, 448.f));
+  const int ex = int((b >> 23) & 0xFFu);
+  const uint32_t man = b & 0x7FFFFFu;
+  int e;
+  if (ex != 0) {
+    e = ex - 127 + (man != 0 ? 1 : 0);
+  } else {  // subnormal ratio: ceil(log2(man * 2^-149))
+    const int top = 31 - __clz(int(man));
+    e = -149 + top + ((man & ((1u << top) - 1u)) != 0 ? 1 : 0);
+  }
+  return min(max(e + 127, 0), 254);
+}
+// 2^-e as float32 for e = code - 127: its biased exponent is 254 - code (code 254 gives the
+// subnormal 2^-127).
+__device__ __forceinline__ float mx_inv_scale(int code) {
+  const int pe = 254 - code;  // in [0, 254]
+  return pe >= 1 ? __uint_as_float(uint32_t(pe) << 23) : __uint_as_float(0x00400000u);  // 2^-127 for pe == 0
+}
+
+// Activations: 4 lanes x 8 bf16 per 32-wide group (quarter-warp shuffles for the amax).
+__global__ void __launch_bounds__(256) quant_act_mx32_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
+                                                             int64_t ld_x, uint8_t* __restrict__ q,
+                                                             uint8_t* __restrict__ ecode) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t G = K / 32;
+  const int64_t total = M * G;  // groups
+  const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthreads = int64_t(gridDim.x) * blockDim.x;
+  // thread -> (group gi = idx / 4, part = idx % 4); every lane of a quarter-warp iterates together
+  for (int64_t idx = tid; idx < (total * 4 + 31) / 32 * 32; idx += nthreads) {
+    const int64_t gi = idx >> 2;
+    const int part = int(idx & 3);
+    const bool valid = gi < total;
+    const int64_t m = valid ? gi / G : 0;
+    const int64_t g = valid ? gi - m * G : 0;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (valid) v = ld_nc_v4(x + m * ld_x + g * 32 + part * 8);
+    float f[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                  bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const int code = mx_code_for_amax(amax);
+    const float inv = mx_inv_scale(code);
+    if (valid) {
+      uint2 out;
+      out.x = cvt4_e4m3(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv), __fmul_rn(f[2], inv), __fmul_rn(f[3], inv));
+      out.y = cvt4_e4m3(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv), __fmul_rn(f[6], inv), __fmul_rn(f[7], inv));
+      *reinterpret_cast<uint2*>(q + m * K + g * 32 + part * 8) = out;
+      if (part == 0) ecode[m * G + g] = uint8_t(code);
+    }
+  }
+}
+
+// Weights: one warp per 32x32 block, lane = row; the block's amax is a warp maximum.
+__global__ void __launch_bounds__(256) quant_weight_mx32_kernel(const float* __restrict__ w, int64_t N, int64_t K,
+                                                                uint8_t* __restrict__ q, uint8_t* __restrict__ ecode) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t G = K / 32, NB = (N + 31) / 32;
+  const int lane = threadIdx.x & 31;
+  const int64_t blk = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (blk >= NB * G) return;
+  const int64_t nb = blk / G, g = blk - nb * G;
+  const int64_t row = nb * 32 + lane;
+  const bool valid = row < N;
+  float4 v[8];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[i] = valid ? __ldg(reinterpret_cast<const float4*>(w + row * K + g * 32) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  const int code = mx_code_for_amax(amax);
+  const float inv = mx_inv_scale(code);
+  if (lane == 0) ecode[nb * G + g] = uint8_t(code);
+  if (!valid) return;
+  uint32_t packed[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    packed[i] = cvt4_e4m3(__fmul_rn(v[i].x, inv), __fmul_rn(v[i].y, inv), __fmul_rn(v[i].z, inv), __fmul_rn(v[i].w, inv));
+  uint4* dst = reinterpret_cast<uint4*>(q + row * K + g * 32);
+  dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+}
+
+int launch_quant_act_mx32(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q, void* ecode, void* stream) {
+  const int64_t threads_needed = M * (K / 32) * 4;
+  const int64_t cap = int64_t(device_sm_count()) * 8;
+  const int blocks = int(std::min<int64_t>((threads_needed + 255) / 256, cap));
+  return launch_kernel(quant_act_mx32_kernel, dim3(std::max(blocks, 1)), dim3(256), 0, stream,
+                       static_cast<const uint16_t*>(x), M, K, ld_x, static_cast<uint8_t*>(q),
+                       static_cast<uint8_t*>(ecode));
+}
+
+int launch_quant_weight_mx32(const float* w, int64_t N, int64_t K, void* q, void* ecode, void* stream) {
+  const int64_t blocks = ((N + 31) / 32) * (K / 32);  // one warp each, 8 per CTA
+  return launch_kernel(quant_weight_mx32_kernel, dim3(unsigned((blocks + 7) / 8)), dim3(256), 0, stream, w, N, K,
+                       static_cast<uint8_t*>(q), static_cast<uint8_t*>(ecode));
 }
 
 int launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ld_x, void* q, float* scale, void* stream) {

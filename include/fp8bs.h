@@ -183,6 +183,39 @@ fp8bs_status fp8bs_gemm_a8w8_blockscale_noalloc(const void* A_e4m3, const float*
                                                 int64_t K, fp8bs_stream_t stream);
 
 /*
+ * MX32 variant ([aiter#7247] ROCm/aiter PR #7247, "Motivation": the 32x32 MXFP8 GEMMs,
+ * w_scale_block 32x32, dense and batched): e4m3 operands with E8M0 scales (one byte, value
+ * 2^(code - 127)) on 32-wide K groups -- per token for activations, per 32x32 block for
+ * weights -- and float32 accumulation:
+ *   out[b,m,n] = sum_g 2^(a_e8m0[b,m,g] - 127) * 2^(w_e8m0[b,n/32,g] - 127)
+ *                      * sum_{k = 32g .. 32g+31} A[b,m,k] * W[b,n,k]
+ * Quantisation: code = clamp(ceil(log2(float32(amax) / 448)) + 127, 0, 254) (0 when amax is
+ * 0; the exponent read exactly from the float32 quotient), q = e4m3_rn_satfinite(x * 2^-e).
+ * The tensor core applies the scales itself (tcgen05.mma kind::mxf8f6f4.block_scale).
+ *
+ * fp8bs_quant_act_mx32: x_bf16 [M, ld_x] (ld_x >= K, ld_x % 8 == 0), K % 32 == 0 ->
+ *   q_e4m3 [M, K], a_e8m0 [M, K/32] (device). Bit-identical to the CPU oracle.
+ * fp8bs_quant_weight_mx32: w_f32 [N, K], K % 32 == 0 -> q_e4m3 [N, K],
+ *   w_e8m0 [ceil(N/32), K/32] (device); a partial last block is quantised over its rows.
+ * fp8bs_gemm_a8w8_mx32: batch >= 1 independent GEMMs on contiguous stacks A_e4m3
+ *   [batch, M, K], a_e8m0 [batch, M, K/32], W_e4m3 [batch, N, K], w_e8m0 [batch,
+ *   ceil(N/32), K/32], out_bf16 [batch, M, N] (batch = 1 is the dense GEMM). Requires
+ *   K % 128 == 0, N % 16 == 0, 16-byte aligned pointers. workspace: at least
+ *   fp8bs_mx32_workspace_bytes(batch, M, N, K) bytes, zero-filled once, as for
+ *   fp8bs_gemm_a8w8_blockscale (split-K arrival counters are left at zero). Results are
+ *   deterministic and within the float32-accumulation bound of the float64 oracle rounded
+ *   once to bf16.
+ */
+fp8bs_status fp8bs_quant_act_mx32(const void* x_bf16, int64_t M, int64_t K, int64_t ld_x, void* q_e4m3,
+                                  uint8_t* a_e8m0, fp8bs_stream_t stream);
+fp8bs_status fp8bs_quant_weight_mx32(const float* w_f32, int64_t N, int64_t K, void* q_e4m3, uint8_t* w_e8m0,
+                                     fp8bs_stream_t stream);
+size_t fp8bs_mx32_workspace_bytes(int64_t batch, int64_t M, int64_t N, int64_t K);
+fp8bs_status fp8bs_gemm_a8w8_mx32(const void* A_e4m3, const uint8_t* a_e8m0, const void* W_e4m3,
+                                  const uint8_t* w_e8m0, void* out_bf16, int64_t batch, int64_t M, int64_t N,
+                                  int64_t K, void* workspace, size_t workspace_bytes, fp8bs_stream_t stream);
+
+/*
  * Companion bf16 GEMM for the small-N router / indexer projections ([cookbook#8]:
  * the live BF16 lookups are the MoE router and the DSA indexer's weights_proj;
  * [aiter#7247] "Technical Details": N = 32..1024, some with fp32 output).

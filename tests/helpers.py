@@ -64,6 +64,33 @@ def check_a8w8(y_bf16: torch.Tensor, A_q, a_s, W_q, w_s, rows=None):
     return rl, ometrics.rel_l2(y, ref_bf16)
 
 
+def check_mx32(y_bf16: torch.Tensor, A_q, a_e, W_q, w_e, rows=None):
+    """Element-wise and relative-L2 parity of a GPU MX32 GEMM output against the MX oracle,
+    with the same bound as the 128-block GEMM: one bf16 rounding plus 2^-12 of the terms'
+    absolute sum (a float32-accumulating tensor core meets it with a wide margin)."""
+    from oracle import mx as omx
+    if rows is not None:
+        A_q, a_e = A_q[rows], a_e[rows]
+    ref, _ = omx.gemm_a8w8_mx32(A_q, a_e, W_q, w_e)
+    y = y_bf16.float().cpu().numpy().astype(np.float64)
+    if rows is not None:
+        y = y[rows]
+    A = np.abs(oe4m3.decode(A_q))
+    W = np.abs(oe4m3.decode(W_q))
+    sa, sw = omx.e8m0_decode(a_e), omx.e8m0_decode(w_e)
+    nb = np.arange(W.shape[0]) // 32
+    asum = np.zeros_like(ref)
+    for g in range(A.shape[1] // 32):
+        ks = slice(32 * g, 32 * g + 32)
+        asum += sa[:, g][:, None] * sw[nb, g][None, :] * (A[:, ks] @ W[:, ks].T)
+    tol = 2.0 ** -8 * np.abs(ref) + 2.0 ** -12 * asum
+    bad = np.abs(y - ref) > tol
+    assert not bad.any(), f"{bad.sum()} of {bad.size} outputs outside the bound"
+    rl = ometrics.rel_l2(y, ref)
+    assert rl <= REL_L2_TOL, rl
+    return rl
+
+
 def check_bf16(y: torch.Tensor, A, W, out_fp32: bool, rows=None):
     A = np.asarray(A, dtype=np.float64)
     W = np.asarray(W, dtype=np.float64)
