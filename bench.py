@@ -20,8 +20,9 @@ has no exchange step).
 
 The default run also measures, with a few steps each, every other configuration: the
 prefill shapes, the dense M ladder (with the dispatch census and its padded-M drift), the
-bf16 small-N GEMMs, the bf16 lm_head and the fused residual add + RMSNorm + quantisation
-step, each as an entry of "workloads" with its own roofline; the
+bf16 small-N GEMMs, the bf16 lm_head, the fused residual add + RMSNorm + quantisation
+step and the MX32 GEMMs (dense and batched), each as an entry of "workloads" with its own
+roofline; the
 per-shape "detail" table gives cold- and hot-weight us/call, and the CPU leg reports the
 oracle's time and the accuracy of the timed outputs against it. --only skips the extra
 workloads.
@@ -840,6 +841,163 @@ def measure_bf16(args, world, rank, dev, steps, warmup, detail, e2e_steps, cpu, 
     return line
 
 
+# --------------------------------------------------------------------------- MX32 workloads
+MX_METRIC = "MX32 a8w8 GEMM µs/call, TFLOPS & HBM GB/s (cold weights) vs roofline"
+
+
+def mx_calls(workload):
+    """(batch, M, N, K) of an MX32 workload."""
+    if workload == "mx32_batched":
+        b, N, K = inputs.MX32_BATCHED
+        return [(b, M, N, K) for M in inputs.MX32_BATCHED_MS]
+    return [(1, M, N, K) for (N, K) in inputs.MX32_NK for M in inputs.MX32_MS]
+
+
+def mx_bytes(b, M, N, K):
+    """A + a_e8m0 + W + w_e8m0 + out."""
+    return b * (M * K + M * (K // 32) + N * K + ((N + 31) // 32) * (K // 32) + 2 * M * N)
+
+
+def measure_mx(args, world, rank, dev, workload, steps, warmup, detail):
+    """An MX32 workload: calls on weights rotated over >= 512 MiB of copies, one CUDA graph
+    per rotation phase (rank 0's line; None elsewhere)."""
+    import torch
+
+    import fp8_block_scaled_a8w8_b200 as fb
+
+    fb.lib()
+    pk = peaks()
+    calls = mx_calls(workload)
+    shapes = sorted({(b, N, K) for (b, M, N, K) in calls})
+    wcopies, acts = {}, {}
+    for si, (b, N, K) in enumerate(shapes):
+        uses = sum(1 for c in calls if (c[0], c[2], c[3]) == (b, N, K))
+        w = inputs.weight_f32(b * N, K, 700 + si).to(dev)
+        wq, we = fb.quant_weight_mx32(w)
+        del w
+        # per batch the 32-row blocks must not straddle batches: N % 32 == 0 for these shapes
+        wq, we = wq.view(b, N, K), we.view(b, (N + 31) // 32, K // 32)
+        per = wq.numel() + we.numel()
+        n = max(1, math.ceil(ROTATE_BYTES / per))
+        n = uses * math.ceil(n / uses)
+        wcopies[(b, N, K)] = [(wq, we)] + [(wq.clone(), we.clone()) for _ in range(n - 1)]
+    for (b, M, N, K) in calls:
+        if (b, M, K) not in acts:
+            x = inputs.activation_bf16(b * M, K, 800 + M + K).to(dev)
+            q, e = fb.quant_act_mx32(x)
+            acts[(b, M, K)] = (q.view(b, M, K) if b > 1 else q, e.view(b, M, K // 32) if b > 1 else e)
+    outs = [torch.empty(((b,) if b > 1 else ()) + (M, N), dtype=torch.bfloat16, device=dev) for (b, M, N, K) in calls]
+    ws = torch.zeros(max(256, max(fb.mx32_workspace_bytes(b, M, N, K) for (b, M, N, K) in calls)), dtype=torch.uint8,
+                     device=dev)
+    period = 1
+    for key, cp in wcopies.items():
+        u = sum(1 for c in calls if (c[0], c[2], c[3]) == key)
+        period = period * (len(cp) // u) // math.gcd(period, len(cp) // u)
+    stream = torch.cuda.Stream(device=dev)
+
+    def weights(s, c):
+        b, M, N, K = calls[c]
+        k = sum(1 for j in range(c) if (calls[j][0], calls[j][2], calls[j][3]) == (b, N, K))
+        u = sum(1 for j in range(len(calls)) if (calls[j][0], calls[j][2], calls[j][3]) == (b, N, K))
+        cp = wcopies[(b, N, K)]
+        wq, we = cp[(s * u + k) % len(cp)]
+        return (wq[0], we[0]) if b == 1 else (wq, we)
+
+    def step(s, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        for c, (b, M, N, K) in enumerate(calls):
+            q, e = acts[(b, M, K)]
+            wq, we = weights(s, c)
+            fb.gemm_a8w8_mx32(q, e, wq, we, out=outs[c], workspace=ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    events = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(period)]
+    graphs = []
+    with torch.cuda.stream(stream):
+        for ph in range(period):
+            step(ph)
+        stream.synchronize()
+        for ph in range(period):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(ph, events[ph])
+            graphs.append(g)
+        for s_ in range(warmup):
+            graphs[s_ % period].replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index)
+    if rank == 0:
+        clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for s_ in range(steps):
+        with torch.cuda.stream(stream):
+            graphs[(warmup + s_) % period].replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop() if rank == 0 else None
+    step_ms = max_over_ranks(t0.elapsed_time(t1) / steps, dev)
+    line = None
+    if rank == 0:
+        gemm_ms = float(np.mean([events[ph][0].elapsed_time(events[ph][1]) for ph in sorted(
+            {(warmup + s_) % period for s_ in range(steps)})]))
+        tot_bytes = float(sum(mx_bytes(*c) for c in calls))
+        tot_flops = float(sum(2.0 * b * M * N * K for (b, M, N, K) in calls))
+        fp8_peak = 2.0 * pk["bf16_tflops_sustained"]
+        t_roof = sum(max(mx_bytes(*c) / (pk["hbm_gbs"] * 1e9), 2.0 * c[0] * c[1] * c[2] * c[3] / (fp8_peak * 1e12))
+                     for c in calls)
+        if tot_bytes / (pk["hbm_gbs"] * 1e9) >= tot_flops / (fp8_peak * 1e12):
+            ach = tot_bytes / (gemm_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(ach / pk["hbm_gbs"], 4)}
+        else:
+            ach = tot_flops / (gemm_ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                    "frac": round(ach / fp8_peak, 4),
+                    "peak_source": "2 x measured sustained bf16 cuBLAS (fp8/bf16 nominal ratio 2)"}
+        roof.update({"roofline_time_frac": round(t_roof / (gemm_ms * 1e-3), 4), "traffic": None,
+                     "kernel": "gemm_mx_kernel (tcgen05.mma kind::mxf8f6f4.block_scale)",
+                     "gemm_us_per_step": round(gemm_ms * 1000.0, 2)})
+        det = None
+        if detail:
+            det = []
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            for c, (b, M, N, K) in enumerate(calls):
+                q, e = acts[(b, M, K)]
+                cp = wcopies[(b, N, K)]
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(stream):
+                    with torch.cuda.graph(g, stream=stream):
+                        for r in range(20):
+                            wq, we = cp[r % len(cp)]
+                            if b == 1:
+                                wq, we = wq[0], we[0]
+                            fb.gemm_a8w8_mx32(q, e, wq, we, out=outs[c], workspace=ws, stream=stream)
+                    ts = []
+                    for _ in range(5):
+                        e0.record(stream)
+                        g.replay()
+                        e1.record(stream)
+                        e1.synchronize()
+                        ts.append(e0.elapsed_time(e1) * 1000.0 / 20)
+                del g
+                us = sorted(ts)[len(ts) // 2]
+                by, fl = mx_bytes(b, M, N, K), 2.0 * b * M * N * K
+                roof_us = max(by / (pk["hbm_gbs"] * 1e3), fl / (2 * pk["bf16_tflops"] * 1e6))
+                det.append({"batch": b, "M": M, "N": N, "K": K, "us": round(us, 3), "GBps": round(by / us / 1e3, 1),
+                            "TFLOPS": round(fl / us / 1e6, 2), "roofline_frac": round(roof_us / us, 3)})
+        line = {"metric": MX_METRIC, "value": round(step_ms * 1000.0 / (len(calls) * world), 3), "unit": "µs/call",
+                "ms_per_step": round(step_ms, 4), "steps": steps, "warmup": warmup, "dtype": "e4m3 x e4m3 (E8M0) -> f32",
+                "config": {"workload": workload, "description": inputs.WORKLOADS[workload], "calls_per_step": len(calls),
+                           "weight_rotation_mib": ROTATE_BYTES >> 20},
+                "roofline": roof, "gpu_launches": len(calls) * steps, "clocks": clk, "detail": det}
+    graphs.clear()
+    return line
+
+
 # --------------------------------------------------------------------------- fused norm + quant workload
 NORM_METRIC = "add_rmsnorm_quant µs/call & HBM GB/s vs roofline"
 
@@ -946,6 +1104,8 @@ def run_reference(args):
         return run_reference_bf16(args, world)
     if args.workload == "add_rmsnorm_quant":
         return run_reference_norm(args, world)
+    if args.workload in ("mx32", "mx32_batched"):
+        return run_reference_mx(args, world)
     calls = workload_calls(args.workload)
     wcache = {}
 
@@ -1001,6 +1161,38 @@ def run_reference_norm(args, world):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_mx(args, world):
+    """The oracle's MX32 quantisation + GEMM, one call per step (M > 64 timed on 64 rows and
+    scaled by M / 64; the batched form timed on one batch and scaled by b)."""
+    from oracle import mx as omx
+    calls = mx_calls(args.workload)
+    wcache = {}
+
+    def one(c):
+        b, M, N, K = calls[c % len(calls)]
+        if (N, K) not in wcache:
+            wcache[(N, K)] = omx.quant_weight_mx32(inputs.weight_f32(N, K, 700).numpy())  # set-up, untimed
+        m = min(M, 64)
+        x = inputs.activation_bf16(m, K, 800 + M + K).float().numpy()
+        t0 = time.perf_counter()
+        Aq, Ae = omx.quant_act_mx32(x)
+        omx.gemm_a8w8_mx32(Aq, Ae, *wcache[(N, K)])
+        return (time.perf_counter() - t0) * b * M / m
+
+    for s in range(args.warmup):
+        one(s)
+    us = float(np.mean([one(args.warmup + s) for s in range(args.steps)])) * 1e6
+    line = {"impl": "reference", "metric": MX_METRIC, "value": round(us, 1), "unit": "µs/call", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(us / 1000.0, 3), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "description": inputs.WORKLOADS[args.workload]},
+            "cpu_baseline": {"value": round(us, 1), "unit": "µs/call", "cores": _threads(), **_host(), "kind": "oracle",
+                             "sample": "one call per step, cycling through the calls; M > 64 timed on 64 rows and "
+                                       "scaled, batches scaled by b"},
+            "e2e": {"value": round(us, 1), "unit": "µs/call", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference_bf16(args, world):
     calls = bf16_calls(args.workload)
     wcache = {}
@@ -1046,6 +1238,8 @@ def run_gpu(args):
                                 args.cpu_baseline, args.workload)
         elif args.workload == "add_rmsnorm_quant":
             line = measure_norm(args, world, rank, dev, args.steps, args.warmup)
+        elif args.workload in ("mx32", "mx32_batched"):
+            line = measure_mx(args, world, rank, dev, args.workload, args.steps, args.warmup, args.detail)
         else:
             line = measure_a8w8(args, world, rank, dev, args.workload, args.shape, args.steps, args.warmup,
                                 args.detail, args.e2e_steps, args.cpu_baseline)
@@ -1064,6 +1258,9 @@ def run_gpu(args):
                 torch.cuda.empty_cache()
             subs["add_rmsnorm_quant"] = measure_norm(args, world, rank, dev, min(args.steps, 20), 3)
             torch.cuda.empty_cache()
+            for w in ("mx32", "mx32_batched"):
+                subs[w] = measure_mx(args, world, rank, dev, w, min(args.steps, 10), 3, True)
+                torch.cuda.empty_cache()
             if rank == 0:
                 line["workloads"] = {w: compact(v) for w, v in subs.items()}
         if rank == 0:

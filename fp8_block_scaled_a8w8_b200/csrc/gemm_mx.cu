@@ -45,7 +45,12 @@ constexpr int kMxStages = 4;
 constexpr int kMxABytes = kMxBM * 128, kMxBBytes = kMxBN * 128, kMxStageBytes = kMxABytes + kMxBBytes;
 constexpr int kMxEpiWarps = 8;
 constexpr int kMxOutBytes = kMxEpiWarps * 2048;  // one 32 x 32 bf16 staging box per epilogue warp
-constexpr size_t kMxSmemBytes = size_t(kMxStages) * kMxStageBytes + kMxOutBytes + 1024 + 256;
+// scale-byte prefetch ring of each scale-factor writer warp: 128 activation-row words +
+// 8 weight-block words per stage, kMxSfAhead stages in flight
+constexpr int kMxSfSlotBytes = 512 + 32;
+constexpr int kMxSfRing = 8, kMxSfAhead = 6;
+constexpr int kMxSfBytes = 4 * kMxSfRing * kMxSfSlotBytes;
+constexpr size_t kMxSmemBytes = size_t(kMxStages) * kMxStageBytes + kMxOutBytes + kMxSfBytes + 1024 + 256;
 constexpr uint32_t kMxSfBase = 2 * kMxBN;  // TMEM: [2 accumulators][scale-factor slots of 32 columns]
 static_assert(kMxSfBase + 32 * kMxStages <= 512, "TMEM budget");
 static_assert(kMxStageBytes % 1024 == 0, "stage alignment");
@@ -158,6 +163,29 @@ __device__ __forceinline__ MxItem mx_item(const MxParams& p, int item) {
   return r;
 }
 
+// Walks this CTA's stages (item, K block) in order.
+struct MxStageIter {
+  MxItem w;
+  int item, kb;
+  bool valid;
+  __device__ MxStageIter(const MxParams& p, int items) : item(blockIdx.x) {
+    valid = item < items;
+    if (valid) {
+      w = mx_item(p, item);
+      kb = w.kb0;
+    }
+  }
+  __device__ void advance(const MxParams& p, int items) {
+    if (++kb < w.kb1) return;
+    item += gridDim.x;
+    valid = item < items;
+    if (valid) {
+      w = mx_item(p, item);
+      kb = w.kb0;
+    }
+  }
+};
+
 template <bool kSplitK>
 __global__ void __launch_bounds__(kMxThreads, 1)
     gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -167,7 +195,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* out_stage = smem + size_t(S) * kMxStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + kMxOutBytes);
+  uint8_t* sf_ring = out_stage + kMxOutBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sf_ring + kMxSfBytes);
   // bars: full[S], empty[S], sf_full[S], tfull[2], tempty[2], drain
   uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
   uint32_t* tmem_slot = misc;
@@ -270,44 +299,67 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ scale-factor writers
-    // warp q writes TMEM lanes 32q..32q+31 (every subpartition holds the same copy)
-    const uint32_t lane_addr = tmem_base + (uint32_t(32 * (warp & 3)) << 16);
-    int it = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
-      const MxItem w = mx_item(p, item);
-      const uint8_t* arow = p.a_e + (int64_t(w.bt) * p.M) * p.K32;
-      const uint8_t* wrow = p.w_e + (int64_t(w.bt) * p.NB32) * p.K32;
-      for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
-        const int s = it % S;
-        // scale bytes of the four K groups of this stage: 4 consecutive bytes per row / block
-        uint32_t sa[4], sb[8];
+    // Warp q writes TMEM lanes 32q..32q+31 (every subpartition holds the same copy). The
+    // scale bytes come from global memory (L2) with a latency of several stages, so each
+    // warp copies them kMxSfAhead stages ahead with cp.async into its own shared-memory
+    // ring: its lanes' 4 activation rows (4 bytes = 4 K groups each) and the tile's 6
+    // weight blocks, one commit group per stage.
+    const int q = warp & 3;
+    const uint32_t lane_addr = tmem_base + (uint32_t(32 * q) << 16);
+    const uint32_t ring = smem_u32(sf_ring + q * kMxSfRing * kMxSfSlotBytes);
+    MxStageIter use_it(p, items), fetch_it(p, items);
+    auto fetch = [&](int slot) {
+      if (fetch_it.valid) {
+        const MxItem& w = fetch_it.w;
+        const uint8_t* arow = p.a_e + (int64_t(w.bt) * p.M) * p.K32 + 4 * fetch_it.kb;
+        const uint8_t* wrow = p.w_e + (int64_t(w.bt) * p.NB32) * p.K32 + 4 * fetch_it.kb;
+        const uint32_t base = ring + slot * kMxSfSlotBytes;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int r = w.tm * kMxBM + lane + 32 * j;
-          sa[j] = r < p.M ? __ldg(reinterpret_cast<const uint32_t*>(arow + int64_t(r) * p.K32 + 4 * kb)) : 0x7F7F7F7Fu;
+          const int r = min(w.tm * kMxBM + lane + 32 * j, p.M - 1);  // rows past M: any valid row
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + 4 * (32 * j + lane)),
+                       "l"(arow + int64_t(r) * p.K32)
+                       : "memory");
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int nb = w.tn * (kMxBN / 32) + j;
-          sb[j] = (j < kMxBN / 32 && nb < p.NB32)
-                      ? __ldg(reinterpret_cast<const uint32_t*>(wrow + int64_t(nb) * p.K32 + 4 * kb))
-                      : 0x7F7F7F7Fu;
+        if (lane < kMxBN / 32) {
+          const int nb = min(w.tn * (kMxBN / 32) + lane, p.NB32 - 1);
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + 512 + 4 * lane),
+                       "l"(wrow + int64_t(nb) * p.K32)
+                       : "memory");
         }
-        if (!__all_sync(0xffffffffu, mx_wait(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, lim))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t slot = lane_addr + kMxSfBase + uint32_t(32 * s);
-        mx_tmem_st_x4(slot, sa[0], sa[1], sa[2], sa[3]);  // column j: rows 32j + lane
-        mx_tmem_st_x8(slot + 16, sb);                      // column j: output columns 32j .. 32j + 31
-        mx_tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sf_full_bar(s));
+        fetch_it.advance(p, items);
       }
+      asm volatile("cp.async.commit_group;" ::: "memory");  // one group per stage, empty past the end
+    };
+#pragma unroll 1
+    for (int d = 0; d < kMxSfAhead; ++d) fetch(d % kMxSfRing);
+    int it = 0;
+    for (; use_it.valid; ++it) {
+      fetch((it + kMxSfAhead) % kMxSfRing);
+      asm volatile("cp.async.wait_group %0;" ::"n"(kMxSfAhead) : "memory");  // stage it's bytes have landed
+      __syncwarp();
+      const int s = it % S;
+      const uint32_t base = ring + (it % kMxSfRing) * kMxSfSlotBytes;
+      uint32_t sa[4], sb[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sa[j]) : "r"(base + 4 * (32 * j + lane)));
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        sb[j] = 0x7F7F7F7Fu;
+        if (j < kMxBN / 32) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sb[j]) : "r"(base + 512 + 4 * j));
+      }
+      if (!__all_sync(0xffffffffu, mx_wait(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, lim))) break;
+      tc_fence_after();
+      const uint32_t slot = lane_addr + kMxSfBase + uint32_t(32 * s);
+      mx_tmem_st_x4(slot, sa[0], sa[1], sa[2], sa[3]);  // column j: rows 32j + lane
+      mx_tmem_st_x8(slot + 16, sb);                      // column j: output columns 32j .. 32j + 31
+      mx_tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sf_full_bar(s));
+      use_it.advance(p, items);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing in flight into the ring at exit
   } else if (warp >= 8) {
     // ------------------------------------------------------------ epilogue warps 8..15
     const int e = warp - 8, q = warp & 3, h = e >> 2;  // lane quarter, 96-column half
@@ -384,16 +436,26 @@ __global__ void __launch_bounds__(kMxThreads, 1)
 #pragma unroll
               for (int j = 0; j < 32; ++j) sum[j] = 0.f;
 #pragma unroll 1
-              for (int sp = 0; sp < p.splits; ++sp) {
-                const float* src = p.part + ((int64_t(w.tile) * p.splits + sp) * kMxBM + 32 * q + lane) * kMxBN +
-                                   h * (kMxBN / 2) + 32 * c;
+              for (int sp0 = 0; sp0 < p.splits; sp0 += 2) {  // two splits' loads in flight (16 x 16 B)
+                float4 f[2][8];
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                  const float4 f = __ldcg(reinterpret_cast<const float4*>(src + j));
-                  sum[j] += f.x;
-                  sum[j + 1] += f.y;
-                  sum[j + 2] += f.z;
-                  sum[j + 3] += f.w;
+                for (int u = 0; u < 2; ++u) {
+                  const int sp = sp0 + u < p.splits ? sp0 + u : sp0;
+                  const float* src = p.part + ((int64_t(w.tile) * p.splits + sp) * kMxBM + 32 * q + lane) * kMxBN +
+                                     h * (kMxBN / 2) + 32 * c;
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) f[u][j] = __ldcg(reinterpret_cast<const float4*>(src + 4 * j));
+                }
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                  if (sp0 + u >= p.splits) break;
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) {
+                    sum[4 * j] += f[u][j].x;
+                    sum[4 * j + 1] += f[u][j].y;
+                    sum[4 * j + 2] += f[u][j].z;
+                    sum[4 * j + 3] += f[u][j].w;
+                  }
                 }
               }
               const int col0 = col_base + 32 * c;

@@ -34,6 +34,12 @@ LADDER_NK = (5120, 6144)
 # small-N bf16 GEMMs: (N, K, fp32 output?)
 BF16_NK = [(256, 6144, False), (32, 6144, False), (384, 5120, False), (1024, 5120, True), (128, 512, False)]
 BF16_MS = [1, 32, 576, 4096, 16384]
+# the MX32 (32x32 E8M0 scale block) GEMMs of [aiter#7247] "Technical Details" and its
+# microbenchmark table: dense (N, K) at M = 48 and 768, batched b = 8 (1024, 4096) at M = 16
+MX32_NK = [(1792, 5120), (4608, 5120), (5120, 2304), (5120, 8192), (32768, 1280)]
+MX32_MS = [48, 768]
+MX32_BATCHED = (8, 1024, 4096)
+MX32_BATCHED_MS = [16, 64]
 # the fused residual add + RMSNorm + quantisation step feeding the decode / prefill GEMMs
 NORM_KS = [5120, 6144]
 NORM_MS = [1, 16, 2048, 8192]
@@ -50,6 +56,9 @@ WORKLOADS = {
     "ladder": "a8w8 blockscale dense M ladder, 512 M drawn from 1..8192 on (N,K)=(5120,6144)",
     "bf16_small_n": "bf16 x bf16 small-N GEMMs, M in {1,32,576,4096,16384} x (N,K) in "
                     "{(256,6144),(32,6144),(384,5120),(1024,5120) fp32 out,(128,512)}",
+    "mx32": "MX32 a8w8 GEMM (E8M0 scales, 1x32 / 32x32 blocks), M in {48,768} x (N,K) in "
+            "{(1792,5120),(4608,5120),(5120,2304),(5120,8192),(32768,1280)}, weights rotated over >= 512 MiB",
+    "mx32_batched": "batched MX32 a8w8 GEMM, b=8, (N,K)=(1024,4096), M in {16,64}, weights rotated over >= 512 MiB",
     "add_rmsnorm_quant": "fused residual add + RMSNorm + 1x128 fp8 quantisation, M in {1,16,2048,8192} x "
                          "K in {5120,6144}",
     "lm_head": "bf16 x bf16 large-N lm_head GEMM, M in {24,384,1536,2304,3072} on (N,K)=(32320,5120), bf16 out",
