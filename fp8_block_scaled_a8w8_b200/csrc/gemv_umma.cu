@@ -89,7 +89,7 @@ constexpr int kGuBarBytes = 512;
 constexpr int kGuScaleBytes = 8 * 1024;
 constexpr size_t kGuSmemBytes = size_t(kGuStages) * kGuStageBytes + kGuBarBytes + kGuScaleBytes + 1024;
 static_assert(kGuStageBytes % 1024 == 0, "stage alignment");
-static_assert((2 * kGuStages + 2 * kGuBufs + kGuIssuers) * 8 + 8 * 4 <= kGuBarBytes, "barrier region (misc: 8 words)");
+static_assert((2 * kGuStages + 2 * kGuBufs + kGuIssuers) * 8 + 13 * 4 <= kGuBarBytes, "barrier region (misc: 13 words)");
 static_assert(kGuBufs % kGuIssuers == 0, "a TMEM buffer always belongs to the same issuer");
 static_assert(kGuIssuers >= 1 && kGuIssuers <= 2, "issuers are lane 0 of warps 1 and 2");
 static_assert(kGuCtasPerSm * (kGuSmemBytes + 1024) <= 233472, "two CTAs must fit an SM's shared memory");
@@ -138,33 +138,53 @@ __device__ __forceinline__ void gu_tmem_ld(uint32_t taddr, uint32_t (&r)[NT]) {
     tmem_ld_32x32b_x32(taddr, r);
 }
 
-// Finish block b if this CTA was its last contributor (arrival count old == contributors
-// - 1): all 256 threads sum the contributors' partials in CTA order, kB contributors'
-// loads in flight at a time, store the bf16 output and reset the block's counter.
-// Thread tid owns weight row tid % 128 and tokens tid / 128 + 2j. Contributor cc > cf
-// started its range inside b (its slot 0); the first contributor cf used slot 0 only if
-// its range started exactly at b's first unit, else b was its last block (slot 1).
+// Split-K finish, by a contributor fixed in advance: block b is finished by the CTA
+// whose range holds b's last unit (cl). For that CTA b is its first block, so a CTA
+// finishes at most one block, and the other contributors cf .. cl - 1 only publish their
+// partial (a release add on the block's counter, no round trip). The finisher waits
+// (bounded) until all of them have arrived, then all 256 threads sum the contributors'
+// partials in CTA order, kB contributors' loads in flight at a time, store the output and
+// reset the counter. Thread tid owns weight row tid % 128 and tokens tid / 128 + 2j.
+// Contributor cc > cf started its range inside b (its slot 0); the first contributor cf
+// used slot 0 only if its range started exactly at b's first unit, else b was its last
+// block (slot 1).
+struct GuFinish {
+  int blk;       // block this CTA finishes, or -1
+  int others;    // contributors before this CTA (cl - cf)
+  int cf;        // first contributor
+  int cf_slot;   // its slot for b
+};
+
+__device__ __forceinline__ GuFinish gu_finish_plan(int64_t cta, int64_t u0, int64_t u1, int64_t U, int64_t Cn,
+                                                   int64_t G) {
+  GuFinish f{-1, 0, 0, 0};
+  const int64_t b = u0 / G;
+  if (b * G < u0 && (b + 1) * G <= u1) {  // starts before this range and ends inside it
+    f.blk = int(b);
+    f.cf = int(gu_cta_of_unit(b * G, U, Cn));
+    f.others = int(cta - f.cf);
+    f.cf_slot = (U * f.cf / Cn >= b * G) ? 0 : 1;
+  }
+  return f;
+}
+
 template <int NT>
-__device__ __forceinline__ void gu_finish_block(const GuParams& p, int b, unsigned old, int64_t U, int64_t Cn,
-                                                int64_t G) {
-  const int64_t cf = gu_cta_of_unit(int64_t(b) * G, U, Cn);
-  const int64_t cl = gu_cta_of_unit(int64_t(b + 1) * G - 1, U, Cn);
-  if (old != unsigned(cl - cf)) return;
-  const int cf_slot = (U * cf / Cn >= int64_t(b) * G) ? 0 : 1;
+__device__ __forceinline__ void gu_finish_block(const GuParams& p, const GuFinish& f) {
   constexpr int kE = NT * kGuRows / kGuThreads;  // elements per thread
-  constexpr int kB = kE >= 16 ? 4 : 8;
+  constexpr int kB = kE >= 16 ? 4 : kE >= 8 ? 6 : 8;
   const int tid = threadIdx.x;
   const int r = tid & (kGuRows - 1);
   const int t0 = tid >> 7;
+  const int cf = f.cf, cl = f.cf + f.others;
   float sum[kE];
 #pragma unroll
   for (int j = 0; j < kE; ++j) sum[j] = 0.f;
-  for (int64_t c0 = cf; c0 <= cl; c0 += kB) {
+  for (int c0 = cf; c0 <= cl; c0 += kB) {
     float v[kB][kE];
 #pragma unroll
     for (int jj = 0; jj < kB; ++jj) {
-      const int64_t cc = c0 + jj;
-      const int64_t sl = 2 * cc + (cc == cf ? cf_slot : 0);
+      const int cc = c0 + jj;
+      const int64_t sl = 2 * cc + (cc == cf ? f.cf_slot : 0);
       const float* src = p.part + sl * (kGuSlots * kGuRows) + r;
 #pragma unroll
       for (int j = 0; j < kE; ++j) {
@@ -177,7 +197,7 @@ __device__ __forceinline__ void gu_finish_block(const GuParams& p, int b, unsign
 #pragma unroll
       for (int j = 0; j < kE; ++j) sum[j] += v[jj][j];
   }
-  const int n = b * kGuRows + r;
+  const int n = f.blk * kGuRows + r;
   if (n < p.N) {
 #pragma unroll
     for (int j = 0; j < kE; ++j) {
@@ -185,7 +205,7 @@ __device__ __forceinline__ void gu_finish_block(const GuParams& p, int b, unsign
       if (t < p.M) gu_put(p, int64_t(t) * p.N + n, sum[j]);
     }
   }
-  if (tid == 0) p.counter[b] = 0u;
+  if (tid == 0) p.counter[f.blk] = 0u;
 }
 
 // NT: token columns the epilogue reads per unit (8, 16 or 32 >= M).
@@ -207,8 +227,9 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
   uint32_t* tmem_slot = misc;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* pend_s = reinterpret_cast<volatile int*>(misc + 2);             // n_pending, block 0, block 1
-  volatile unsigned* red_slot = reinterpret_cast<volatile unsigned*>(misc + 5);  // [2]
   volatile int* passed = reinterpret_cast<volatile int*>(misc + 7);  // units whose full-barrier wait has passed
+  volatile int* plan_s = reinterpret_cast<volatile int*>(misc + 8);   // GuFinish: blk, others, cf, cf_slot
+  volatile int* fin_ok = reinterpret_cast<volatile int*>(misc + 12);
   float* sa_s = reinterpret_cast<float*>(smem + size_t(S) * kGuStageBytes + kGuBarBytes);  // [G][NT]
 
   pdl_trigger();
@@ -369,6 +390,15 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
           }
       }
     }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ split-K plan (off the tail)
+    if (lane == 0) {
+      const GuFinish f = gu_finish_plan(cta, u0, u1, U, Cn, G);
+      plan_s[0] = f.blk;
+      plan_s[1] = f.others;
+      plan_s[2] = f.cf;
+      plan_s[3] = f.cf_slot;
+    }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue warps 4..7
     const int q = warp - 4;
@@ -490,15 +520,27 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
     tmem_dealloc(tmem_base, kGuTmemCols);
   }
   pdl_wait();  // warps 1..3 have not waited yet; they write the workspace and the output below
+  if (*abort_flag) return;
+  const GuFinish f{plan_s[0], plan_s[1], plan_s[2], plan_s[3]};
+  // publish the partial sums of the blocks this CTA does not finish (at most two)
   const int n_pending = pend_s[0];
-  const bool aborted = *abort_flag != 0;
-  if (threadIdx.x < n_pending)
-    red_slot[threadIdx.x] = aborted ? 0u : atom_add_acq_rel_gpu(p.counter + pend_s[1 + threadIdx.x], 1u);
-  __syncthreads();
-  if (!aborted) {
-    if (n_pending > 0) gu_finish_block<NT>(p, pend_s[1], red_slot[0], U, Cn, G);
-    if (n_pending > 1) gu_finish_block<NT>(p, pend_s[2], red_slot[1], U, Cn, G);
+  if (threadIdx.x < n_pending && pend_s[1 + threadIdx.x] != f.blk)
+    red_add_release_gpu(p.counter + pend_s[1 + threadIdx.x], 1u);
+  if (f.blk < 0) return;
+  if (threadIdx.x == 0) {  // bounded wait for the other contributors
+    bool ok = true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (ld_acquire_gpu(p.counter + f.blk) != unsigned(f.others)) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&g_status, kStatusTimeout);
+        ok = false;
+        break;
+      }
+    }
+    *fin_ok = ok;
   }
+  __syncthreads();
+  if (*fin_ok) gu_finish_block<NT>(p, f);
 }
 
 // ---------------------------------------------------------------- host side

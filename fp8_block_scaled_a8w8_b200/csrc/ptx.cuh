@@ -239,6 +239,19 @@ __device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v
   return old;
 }
 
+// Arrival without a return value: after a CTA barrier, one thread's release publishes
+// every CTA thread's earlier stores; the arriving CTA does not wait for the round trip.
+__device__ __forceinline__ void red_add_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Acquire load at gpu scope: the stores published by the releases it observes are
+// visible to this thread, and to the CTA after the next barrier.
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // ---------------------------------------------------------------- global loads
 // Streaming 16-byte load: read-only, no L1 allocation, ask L2 to fetch the 256-byte block.
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
