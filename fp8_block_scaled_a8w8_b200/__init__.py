@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "lib", "Fp8bsError", "quant_act_per_token_group", "quant_weight_block128", "gemm_a8w8_blockscale",
     "gemm_bf16", "workspace_bytes", "Workspace", "dispatch_lookup", "dispatch_set_row", "dispatch_reset_table",
-    "dispatch_list_configs", "dispatch_stats", "dispatch_reset_stats", "dispatch_dump_json", "dispatch_table_hash",
+    "dispatch_list_configs", "dispatch_stats", "dispatch_reset_stats", "dispatch_dump_json", "dispatch_dump_table", "dispatch_table_hash",
     "get_device_status", "status_string", "version", "OP_A8W8_BLOCKSCALE", "OP_BF16", "LIB_PATH",
     "FLAG_STATIC_WEIGHTS", "gemm_a8w8_blockscale_noalloc", "test_set_wait_fault", "add_rmsnorm_quant",
     "quant_act_mx32", "quant_weight_mx32", "gemm_a8w8_mx32", "mx32_workspace_bytes",
@@ -69,6 +69,7 @@ _PROTOS = {
                                     ctypes.POINTER(_u64)]),
     "fp8bs_dispatch_reset_stats": (_int, []),
     "fp8bs_dispatch_dump_json": (_int, [ctypes.c_char_p, _sz]),
+    "fp8bs_dispatch_dump_table_json": (_int, [ctypes.c_char_p, _sz]),
     "fp8bs_dispatch_table_hash": (_u64, []),
     "fp8bs_get_device_status": (_int, [_c_void_p]),
     "fp8bs_test_set_wait_fault": (_int, [_u64, _i64]),
@@ -397,6 +398,19 @@ def dispatch_dump_json() -> list:
             return json.loads(buf.value.decode())
         if size > (1 << 28):
             _check("fp8bs_dispatch_dump_json", st)
+        size *= 4
+
+
+def dispatch_dump_table() -> list:
+    """The current table rows: dicts with op, M, N, K, cfg and tuned (chosen by measurement)."""
+    size = 1 << 16
+    while True:
+        buf = ctypes.create_string_buffer(size)
+        st = lib().fp8bs_dispatch_dump_table_json(buf, size)
+        if st == 0:
+            return json.loads(buf.value.decode())
+        if size > (1 << 28):
+            _check("fp8bs_dispatch_dump_table_json", st)
         size *= 4
 
 

@@ -34,6 +34,13 @@ static const KernelConfig kConfigs[] = {
     {"a8w8_tc_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTc, 256, 0, 0},
     {"a8w8_tcw_bn128", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 128, 0, 0},
     {"a8w8_tcw_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 256, 0, 0},
+    // fixed K splits for the tuner (mid M, where the tiles leave SMs idle)
+    {"a8w8_tcw_bn128_sk2", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 128, 2, 0},
+    {"a8w8_tcw_bn128_sk4", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 128, 4, 0},
+    {"a8w8_tcw_bn128_sk6", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 128, 6, 0},
+    {"a8w8_tcw_bn128_sk8", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 128, 8, 0},
+    {"a8w8_tcw_bn256_sk2", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 256, 2, 0},
+    {"a8w8_tcw_bn256_sk4", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcWide, 256, 4, 0},
     {"a8w8_tc2_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcPair, 256, 1, 1},   // depth: MMA halves per K step
     {"a8w8_tc2h_bn256", FP8BS_OP_A8W8_BLOCKSCALE, kPathTcPair, 256, 1, 2},
     {"bf16_gemv_d2", FP8BS_OP_BF16, kPathGemv, 0, 1, 2},
@@ -122,16 +129,29 @@ using CensusKey = std::tuple<int, int64_t, int64_t, int64_t, int64_t, std::strin
 struct State {
   std::mutex mu;
   std::map<Key, const KernelConfig*> rows;
+  std::map<Key, bool> tuned;  // rows whose configuration was chosen by measurement
   std::map<CensusKey, uint64_t> census;
   uint64_t hits[FP8BS_NUM_OPS] = {0, 0};
   uint64_t misses[FP8BS_NUM_OPS] = {0, 0};
   bool log = false;
 };
 
-void add_builtin_rows(std::map<Key, const KernelConfig*>& rows) {
+// Rows chosen by measurement (written by the package's tune.py on a B200): each names the
+// fastest configuration among those that run the shape, timed on cold weights.
+struct TunedRow {
+  int op;
+  int64_t M, N, K;
+  const char* cfg;
+};
+static const TunedRow kTunedRows[] = {
+#include "tuned_rows.inc"
+    {0, 0, 0, 0, nullptr},  // end
+};
+
+void add_builtin_rows(std::map<Key, const KernelConfig*>& rows, std::map<Key, bool>& tuned) {
   // Rows for the decode / prefill projections at the tuner's M ladder: powers of two,
-  // multiples of 16 up to 256. The configuration named is the measured choice for
-  // the shape where one has been made, else the default heuristic.
+  // multiples of 16 up to 256. Each carries the measured choice where the tuner has
+  // timed the shape, else the default heuristic.
   const int64_t nk[][2] = {{5120, 6144}, {14336, 5120}, {16384, 5120}, {34816, 5120}};
   std::vector<int64_t> ms = {1, 2, 4, 8};
   for (int64_t m = 16; m <= 256; m += 16) ms.push_back(m);
@@ -145,12 +165,19 @@ void add_builtin_rows(std::map<Key, const KernelConfig*>& rows) {
     for (int64_t m : bms) rows[Key{FP8BS_OP_BF16, m, p[0], p[1]}] = default_config(FP8BS_OP_BF16, m, p[0], p[1]);
   for (int64_t m : {32, 512, 1024, 2048, 4096})  // lm_head (N = 32320, K = 5120) at the power-of-two ladder
     rows[Key{FP8BS_OP_BF16, m, 32320, 5120}] = default_config(FP8BS_OP_BF16, m, 32320, 5120);
+  for (const auto& r : kTunedRows) {
+    if (!r.cfg) continue;
+    if (const KernelConfig* c = find_config(r.op, r.cfg)) {
+      rows[Key{r.op, r.M, r.N, r.K}] = c;
+      tuned[Key{r.op, r.M, r.N, r.K}] = true;
+    }
+  }
 }
 
 State& state() {
   static State* s = [] {
     auto* st = new State();
-    add_builtin_rows(st->rows);
+    add_builtin_rows(st->rows, st->tuned);
     const char* e = std::getenv("FP8BS_LOG_DISPATCH");
     st->log = e && e[0] == '1';
     return st;
@@ -234,6 +261,7 @@ __attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_set_row(int o
   State& st = state();
   std::lock_guard<std::mutex> lk(st.mu);
   st.rows[Key{op, M, N, K}] = c;
+  st.tuned.erase(Key{op, M, N, K});
   return FP8BS_OK;
 }
 
@@ -241,7 +269,8 @@ __attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_reset_table(i
   State& st = state();
   std::lock_guard<std::mutex> lk(st.mu);
   st.rows.clear();
-  if (keep_builtin) add_builtin_rows(st.rows);
+  st.tuned.clear();
+  if (keep_builtin) add_builtin_rows(st.rows, st.tuned);
   return FP8BS_OK;
 }
 
@@ -301,6 +330,32 @@ __attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_dump_json(cha
                     first ? "" : ",", std::get<0>(k), (long long)std::get<1>(k), (long long)std::get<2>(k),
                     (long long)std::get<3>(k), (long long)std::get<4>(k), std::get<4>(k) ? "true" : "false",
                     std::get<5>(k).c_str(), (unsigned long long)kv.second);
+      s += line;
+      first = false;
+    }
+  }
+  s += "]";
+  if (s.size() >= len) {
+    buf[0] = 0;
+    return FP8BS_ERR_INVALID_ARG;
+  }
+  std::memcpy(buf, s.c_str(), s.size() + 1);
+  return FP8BS_OK;
+}
+
+__attribute__((visibility("default"))) fp8bs_status fp8bs_dispatch_dump_table_json(char* buf, size_t len) {
+  if (!buf || !len) return FP8BS_ERR_INVALID_ARG;
+  State& st = state();
+  std::string s = "[";
+  {
+    std::lock_guard<std::mutex> lk(st.mu);
+    bool first = true;
+    char line[256];
+    for (const auto& kv : st.rows) {
+      const auto& k = kv.first;
+      std::snprintf(line, sizeof line, "%s{\"op\":%d,\"M\":%lld,\"N\":%lld,\"K\":%lld,\"cfg\":\"%s\",\"tuned\":%s}",
+                    first ? "" : ",", std::get<0>(k), (long long)std::get<1>(k), (long long)std::get<2>(k),
+                    (long long)std::get<3>(k), kv.second->name, st.tuned.count(k) ? "true" : "false");
       s += line;
       first = false;
     }

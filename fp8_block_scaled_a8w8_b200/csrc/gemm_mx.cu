@@ -510,7 +510,9 @@ static int mx_splits(int64_t batch, int64_t M, int64_t N, int64_t K) {
   const int64_t kb = K / 128;
   const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + kMxBN - 1) / kMxBN);
   const int64_t sms = device_sm_count();
-  int64_t sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({(sms + tiles - 1) / tiles, kb / 2, 16});
+  // one wave (tiles x splits <= SMs), and at most 4 splits: one CTA sums a tile's partials
+  // (two splits' loads in flight), so each further split adds a round trip to the finish
+  int64_t sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({sms / tiles, kb / 2, 4});
   sp = std::max<int64_t>(1, std::min(sp, kb));
   if (sp > 1 && tiles > kMaxCounters) sp = 1;
   return int(sp);

@@ -499,7 +499,8 @@ static int tc_splits(const KernelConfig& cfg, int64_t M, int64_t N, int64_t K, b
   int64_t sp = cfg.split_k;
   if (sp <= 0) {
     const int64_t sms = device_sm_count();
-    sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({(sms + tiles - 1) / tiles, kb / 2, 8});
+    // one wave: tiles x splits <= SMs (a second, partial wave would double the time)
+    sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({sms / tiles, kb / 2, 8});
   }
   sp = std::max<int64_t>(1, std::min(sp, kb));
   if (sp > 1 && tiles > kMaxCounters) sp = 1;

@@ -350,6 +350,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
     }
   } else if (warp >= 1 && warp <= kGuIssuers) {
     // ------------------------------------------------------------ MMA issuers
+    pdl_wait();  // the bounded waits below start once the previous kernel has completed
     if (lane == 0) {
       const int me = warp - 1;
       bool issued = false;
@@ -519,7 +520,7 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
     tc_fence_after();
     tmem_dealloc(tmem_base, kGuTmemCols);
   }
-  pdl_wait();  // warps 1..3 have not waited yet; they write the workspace and the output below
+  pdl_wait();  // warp 3 has not waited yet; the tail writes the workspace and the output
   if (*abort_flag) return;
   const GuFinish f{plan_s[0], plan_s[1], plan_s[2], plan_s[3]};
   // publish the partial sums of the blocks this CTA does not finish (at most two)

@@ -262,6 +262,12 @@ fp8bs_status fp8bs_dispatch_reset_stats(void);
 /* Census: one JSON object per distinct lookup key with its count, as a JSON array. */
 fp8bs_status fp8bs_dispatch_dump_json(char* buf, size_t len);
 
+/* The current table rows, one JSON object {"op","M","N","K","cfg","tuned"} per row, as a
+ * JSON array ("tuned": the row's configuration was chosen by measurement, see the
+ * package's tune.py; else it is the per-shape default). FP8BS_ERR_INVALID_ARG if len is
+ * too small (buf then holds ""). */
+fp8bs_status fp8bs_dispatch_dump_table_json(char* buf, size_t len);
+
 /* 64-bit FNV-1a hash of the current table rows (identifies the table that ran). */
 uint64_t fp8bs_dispatch_table_hash(void);
 

@@ -3,7 +3,8 @@
 Restates the documented policy in Python and checks the library's choices against it:
 M <= 32 runs the weight-streaming kernel; otherwise the tiled kernel takes the widest tile
 whose output tiles give at least half of the SMs a tile, and splits K (workspace > 0)
-only when even the narrowest tile leaves that many SMs idle. Without a
+only when even the narrowest tile leaves that many SMs idle, into as many splits as keep
+the tiles x splits work items within one wave of SMs. Without a
 GPU the library assumes 148 SMs (B200).
 """
 
@@ -29,7 +30,7 @@ def _splits(M, N, K, bn, kb):
     tiles = math.ceil(M / 128) * math.ceil(N / bn)
     if 2 * tiles >= SMS:
         return 1
-    return max(1, min(math.ceil(SMS / tiles), kb // 2, 8, kb))
+    return max(1, min(SMS // tiles, kb // 2, 8, kb))  # one wave: tiles x splits <= SMs
 
 
 @pytest.mark.parametrize("M", [33, 64, 100, 128, 256, 300, 565, 1099, 2048, 8192])
