@@ -386,7 +386,8 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
                     "peak_source": f"2 x {pk['source']} sustained bf16 cuBLAS (fp8/bf16 nominal ratio 2)"}
         key = "gemv_tma" if all(c == "a8w8_gemv_tma" for c in cfgs) else \
             "gemv_umma" if all(c == "a8w8_gemv_umma" for c in cfgs) else \
-            "gemm_tc" if all(c.startswith("a8w8_tc") for c in cfgs) else None
+            "gemm_fp8" if all(c.startswith(("a8w8_tcw", "a8w8_tc2")) for c in cfgs) else \
+            "gemm_tc" if all(c.startswith("a8w8_tc_") for c in cfgs) else None
         roof["traffic"] = measured_traffic(key, tot_bytes / n_calls) if key else None
         roof["traffic_note"] = "DRAM bytes per launch (average call), ncu capture in profiles/ scaled by algorithmic bytes"
         roof["kernel"] = "gemm_a8w8_blockscale: " + ", ".join(sorted(set(cfgs)))
