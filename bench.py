@@ -203,6 +203,8 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
     fb.lib()
     pk = peaks()
     calls = workload_calls(workload, shape)
+    tiled = getattr(args, "layout", "tiled") == "tiled"
+    tkw = (lambda N: {"tiled_weights": True, "N": N}) if tiled else (lambda N: {})
     if getattr(args, "config", None):  # force one kernel configuration (a table row per call shape)
         for (M, N, K, *_r) in calls:
             fb.dispatch_set_row(fb.OP_A8W8_BLOCKSCALE, M, N, K, args.config)
@@ -217,7 +219,9 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
         w = inputs.weight_f32(N, K, inputs.decode_seed_w(nk_index)).to(dev)
         wq, ws = fb.quant_weight_block128(w)
         del w
-        per = N * K + ws.numel() * 4
+        if tiled:  # the weights stored in 16 KiB tiles (set-up, like the quantisation)
+            wq = fb.tile_weight(wq)
+        per = wq.numel() + ws.numel() * 4
         n = max(1, math.ceil(ROTATE_BYTES / per))
         n = u * math.ceil(n / u)  # a multiple of the uses per step: every step has the same period
         copies = [(wq, ws)] + [(wq.clone(), ws.clone()) for _ in range(n - 1)]
@@ -273,7 +277,7 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
             cp = wcopies[(N, K)]
             wq, wsc = cp[(s * uses[(N, K)] + k) % len(cp)]
             fb.gemm_a8w8_blockscale(qs[c], ss[c], wq, wsc, out=outs[c], workspace=workspace, stream=stream,
-                                    static_weights=True)
+                                    static_weights=True, **tkw(N))
         if ev is not None:
             ev[1].record(stream)
 
@@ -349,7 +353,7 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
                     wq, wsc = cp[(s * uses[(N, K)] + k) % len(cp)]
                     q, sc = fb.quant_act_per_token_group(dx[c], q=qs[c], scale=ss[c], stream=stream)
                     fb.gemm_a8w8_blockscale(q, sc, wq, wsc, out=outs[c], workspace=workspace, stream=stream,
-                                            static_weights=True)
+                                            static_weights=True, **tkw(N))
                     hy[c].copy_(outs[c], non_blocking=True)
         for s in range(3):
             e2e_step(s)
@@ -367,7 +371,7 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
                "api": "fp8_block_scaled_a8w8_b200.quant_act_per_token_group + gemm_a8w8_blockscale (eager)"}
 
     if rank == 0:
-        det = per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk) \
+        det = per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk, tkw=tkw) \
             if detail else None
         tot_bytes = float(sum(a8w8_bytes(M, N, K) for (M, N, K, *_r) in calls))
         tot_ms = gemm_ms_per_call * n_calls
@@ -410,7 +414,7 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
                 wq0, ws0 = wcopies[(N, K)][0]
                 with torch.cuda.stream(stream):
                     q, sc = fb.quant_act_per_token_group(xs[c], stream=stream)
-                    y = fb.gemm_a8w8_blockscale(q, sc, wq0, ws0, workspace=workspace, stream=stream)
+                    y = fb.gemm_a8w8_blockscale(q, sc, wq0, ws0, workspace=workspace, stream=stream, **tkw(N))
                 stream.synchronize()
                 return y.float().cpu().numpy().astype(np.float64)[rows]
             cpu_line = cpu_baseline(workload, calls, [x.cpu() for x in xs], gpu_output)
@@ -423,6 +427,7 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
                        "description": inputs.WORKLOADS[workload] if not shape else "one a8w8 call shape M,N,K",
                        "calls_per_step": n_calls,
                        "weight_rotation_mib": ROTATE_BYTES >> 20,
+                       "weight_layout": "16 KiB tiles (tile_weight)" if tiled else "[N, K] row-major",
                        "l2": "working set per step >> 126 MB L2 (rotated weights); no flush needed",
                        "parallelism": f"replicas x{world}", "timing": "CUDA graphs replayed, CUDA events, max over ranks"},
             "roofline": roof, "quant_roofline": quant_roof,
@@ -456,7 +461,8 @@ def measure_a8w8(args, world, rank, dev, workload, shape, steps, warmup, detail,
     return line
 
 
-def per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk, R=20, rounds=7):
+def per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, stream, pk, R=20, rounds=7,
+                    tkw=lambda N: {}):
     """us/call of every distinct call shape: R back-to-back calls in one CUDA graph, median
     over rounds interleaved across shapes ([aiter#7752] "Kernel": graph replay, median of
     interleaved rounds), once on weight copies rotated over >= 512 MiB (cold: every call
@@ -477,7 +483,7 @@ def per_call_detail(fb, torch, calls, cfgs, wcopies, qs, ss, outs, workspace, st
                     for r in range(R):
                         wq, wsc = cp[r % len(cp)] if kind == "cold" else cp[0]
                         fb.gemm_a8w8_blockscale(qs[c], ss[c], wq, wsc, out=outs[c], workspace=workspace,
-                                                stream=stream, static_weights=True)
+                                                stream=stream, static_weights=True, **tkw(N))
                 graphs[(c, kind)] = g
     times = {k: [] for k in graphs}
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -1279,6 +1285,8 @@ def main():
     ap.add_argument("--workload", default="decode_sweep", choices=list(inputs.WORKLOADS))
     ap.add_argument("--impl", default="fp8bs", choices=["fp8bs", "reference"])
     ap.add_argument("--shape", default=None, help="M,N,K: time one a8w8 call shape instead of a workload")
+    ap.add_argument("--layout", choices=["tiled", "standard"], default="tiled",
+                    help="a8w8 weight storage: 16 KiB tiles (tile_weight, the default) or [N, K] row-major")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-detail", dest="detail", action="store_false",

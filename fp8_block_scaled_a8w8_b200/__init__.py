@@ -21,7 +21,7 @@ __all__ = [
     "gemm_bf16", "workspace_bytes", "Workspace", "dispatch_lookup", "dispatch_set_row", "dispatch_reset_table",
     "dispatch_list_configs", "dispatch_stats", "dispatch_reset_stats", "dispatch_dump_json", "dispatch_dump_table", "dispatch_table_hash",
     "get_device_status", "status_string", "version", "OP_A8W8_BLOCKSCALE", "OP_BF16", "LIB_PATH",
-    "FLAG_STATIC_WEIGHTS", "gemm_a8w8_blockscale_noalloc", "test_set_wait_fault", "add_rmsnorm_quant",
+    "FLAG_STATIC_WEIGHTS", "FLAG_TILED_WEIGHTS", "tile_weight", "tiled_weight_bytes", "gemm_a8w8_blockscale_noalloc", "test_set_wait_fault", "add_rmsnorm_quant",
     "quant_act_mx32", "quant_weight_mx32", "gemm_a8w8_mx32", "mx32_workspace_bytes",
 ]
 
@@ -56,6 +56,8 @@ _PROTOS = {
                                           _c_void_p, _sz, _c_void_p]),
     "fp8bs_gemm_a8w8_blockscale_ex": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i64,
                                              _c_void_p, _sz, ctypes.c_uint32, _c_void_p]),
+    "fp8bs_tiled_weight_bytes": (_sz, [_i64, _i64]),
+    "fp8bs_tile_weight_e4m3": (_int, [_c_void_p, _i64, _i64, _c_void_p, _c_void_p]),
     "fp8bs_gemm_a8w8_blockscale_noalloc": (_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i64, _i64,
                                                   _i64, _c_void_p]),
     "fp8bs_gemm_bf16": (_int, [_c_void_p, _c_void_p, _c_void_p, _int, _i64, _i64, _i64, _c_void_p, _sz, _c_void_p]),
@@ -285,19 +287,45 @@ def _workspace_for(device, nbytes: int):
 
 # ------------------------------------------------------------------ GEMMs
 FLAG_STATIC_WEIGHTS = 1
+FLAG_TILED_WEIGHTS = 2
+
+
+def tiled_weight_bytes(N: int, K: int) -> int:
+    return int(lib().fp8bs_tiled_weight_bytes(N, K))
+
+
+def tile_weight(W: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The tiled copy of e4m3 weight codes W [N, K] (fp8bs_tile_weight_e4m3): 16 KiB tiles,
+    one per 128-row block and 128-wide K group, for gemm_a8w8_blockscale(tiled_weights=True)."""
+    if not _is_byte(W) or W.dim() != 2 or not W.is_contiguous():
+        raise ValueError("W must be a contiguous 2-D one-byte (e4m3 code) tensor")
+    N, K = W.shape
+    nbytes = tiled_weight_bytes(N, K)
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    _check("fp8bs_tile_weight_e4m3", lib().fp8bs_tile_weight_e4m3(_ptr(W), N, K, _ptr(out), _stream(stream)))
+    return out
 
 
 def gemm_a8w8_blockscale(A: torch.Tensor, a_scale: torch.Tensor, W: torch.Tensor, w_scale: torch.Tensor,
                          out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None,
-                         static_weights: bool = False):
+                         static_weights: bool = False, tiled_weights: bool = False, N: int | None = None):
     """out[M, N] bf16 = sum_g a_scale[m,g] w_scale[n/128,g] sum_{k in g} A[m,k] W[n,k] (see include/fp8bs.h).
 
     static_weights: promise that W / w_scale are not written by a kernel still running when
-    this call starts (FP8BS_FLAG_STATIC_WEIGHTS); lets the weight stream start early."""
-    if not (_is_byte(A) and _is_byte(W)) or A.dim() != 2 or W.dim() != 2:
+    this call starts (FP8BS_FLAG_STATIC_WEIGHTS); lets the weight stream start early.
+    tiled_weights: W is the tiled copy from tile_weight() (FP8BS_FLAG_TILED_WEIGHTS); N must
+    then be given."""
+    if not (_is_byte(A) and _is_byte(W)) or A.dim() != 2 or (W.dim() != 2 and not tiled_weights):
         raise ValueError("A and W must be 2-D one-byte (e4m3 code) tensors")
     M, K = A.shape
-    N = W.shape[0]
+    if tiled_weights:
+        if N is None:
+            raise ValueError("tiled_weights needs N")
+        if W.numel() < tiled_weight_bytes(N, K):
+            raise ValueError("W is smaller than the tiled layout of [N, K]")
+    else:
+        N = W.shape[0]
     for t in (A, W, a_scale, w_scale):
         if not t.is_contiguous():
             raise ValueError("operands must be contiguous")
@@ -308,10 +336,11 @@ def gemm_a8w8_blockscale(A: torch.Tensor, a_scale: torch.Tensor, W: torch.Tensor
         workspace = _workspace_for(A.device, need)
     ws_ptr = _ptr(workspace) if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    if static_weights:
+    flags = (FLAG_STATIC_WEIGHTS if static_weights else 0) | (FLAG_TILED_WEIGHTS if tiled_weights else 0)
+    if flags:
         _check("fp8bs_gemm_a8w8_blockscale_ex",
                lib().fp8bs_gemm_a8w8_blockscale_ex(_ptr(A), _ptr(a_scale), _ptr(W), _ptr(w_scale), _ptr(out), M, N, K,
-                                                   ws_ptr, ws_len, FLAG_STATIC_WEIGHTS, _stream(stream)))
+                                                   ws_ptr, ws_len, flags, _stream(stream)))
     else:
         _check("fp8bs_gemm_a8w8_blockscale",
                lib().fp8bs_gemm_a8w8_blockscale(_ptr(A), _ptr(a_scale), _ptr(W), _ptr(w_scale), _ptr(out), M, N, K,

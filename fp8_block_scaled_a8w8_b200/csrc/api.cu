@@ -9,6 +9,8 @@
 #include <set>
 #include <utility>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -170,7 +172,10 @@ FP8BS_API size_t fp8bs_workspace_bytes(int op, int64_t M, int64_t N, int64_t K) 
   int64_t pm = 0;
   bool hit = false;
   const KernelConfig* cfg = dispatch(op, M, N, K, false, &pm, &hit);
-  return cfg ? op_workspace(op, M, N, K, *cfg) : 0;
+  if (!cfg) return 0;
+  // also enough for the shape's default configuration, which a tiled-weight call runs when
+  // the row names a kernel that does not read weight tiles
+  return std::max(op_workspace(op, M, N, K, *cfg), op_workspace(op, M, N, K, *default_config(op, M, N, K)));
 }
 
 static fp8bs_status check_gemm_shape(int64_t M, int64_t N, int64_t K, int64_t kdiv) {
@@ -183,7 +188,7 @@ FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const f
                                                      const float* w_scale, void* out_bf16, int64_t M, int64_t N,
                                                      int64_t K, void* workspace, size_t workspace_bytes, uint32_t flags,
                                                      fp8bs_stream_t stream) {
-  if (flags & ~uint32_t(FP8BS_FLAG_STATIC_WEIGHTS)) return FP8BS_ERR_INVALID_ARG;
+  if (flags & ~uint32_t(FP8BS_FLAG_STATIC_WEIGHTS | FP8BS_FLAG_TILED_WEIGHTS)) return FP8BS_ERR_INVALID_ARG;
   if (!A_e4m3 || !a_scale || !W_e4m3 || !w_scale || !out_bf16) return FP8BS_ERR_INVALID_ARG;
   fp8bs_status st = check_gemm_shape(M, N, K, 128);
   if (st != FP8BS_OK) return st;
@@ -195,6 +200,13 @@ FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const f
   bool hit = false;
   const KernelConfig* cfg = dispatch(FP8BS_OP_A8W8_BLOCKSCALE, M, N, K, true, &pm, &hit);
   if (!cfg) return FP8BS_ERR_UNSUPPORTED;
+  const bool tiled = (flags & FP8BS_FLAG_TILED_WEIGHTS) != 0;
+  if (tiled) {
+    // only the tcgen05 weight-streaming and wide-epilogue kernels read weight tiles: a row
+    // naming another configuration runs the shape's default instead
+    if (cfg->path != kPathGemvUmma && cfg->path != kPathTcWide) cfg = default_config(FP8BS_OP_A8W8_BLOCKSCALE, M, N, K);
+    if (cfg->path == kPathGemvUmma && !gemv_umma_reads_tiles(M, N, K)) return FP8BS_ERR_UNSUPPORTED;
+  }
   const size_t need = op_workspace(FP8BS_OP_A8W8_BLOCKSCALE, M, N, K, *cfg);
   if (need && (!workspace || workspace_bytes < need)) return FP8BS_ERR_WORKSPACE;
   if (need && !aligned16(workspace)) return FP8BS_ERR_ALIGNMENT;
@@ -206,14 +218,28 @@ FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const f
                              (flags & FP8BS_FLAG_STATIC_WEIGHTS) ? 1 : 0, stream);
   else if (cfg->path == kPathGemvUmma)
     e = launch_gemv_umma_a8w8(A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace,
-                              (flags & FP8BS_FLAG_STATIC_WEIGHTS) ? 1 : 0, stream);
+                              (flags & FP8BS_FLAG_STATIC_WEIGHTS) ? 1 : 0, stream, tiled);
   else if (cfg->path == kPathTcWide)
-    e = launch_fp8_tc(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream);
+    e = launch_fp8_tc(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream, tiled);
   else if (cfg->path == kPathTcPair)
     e = launch_fp8_pair(cfg->gemv_depth, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, stream);
   else
     e = launch_tc_a8w8(*cfg, A_e4m3, a_scale, W_e4m3, w_scale, out_bf16, M, N, K, workspace, stream);
   return from_cuda(e);
+}
+
+FP8BS_API size_t fp8bs_tiled_weight_bytes(int64_t N, int64_t K) {
+  if (N <= 0 || K <= 0 || K % 128 != 0) return 0;
+  return tiled_weight_bytes(N, K);
+}
+
+FP8BS_API fp8bs_status fp8bs_tile_weight_e4m3(const void* W_e4m3, int64_t N, int64_t K, void* W_tiled,
+                                              fp8bs_stream_t stream) {
+  if (!W_e4m3 || !W_tiled || N <= 0 || K <= 0 || K % 128 != 0) return FP8BS_ERR_INVALID_ARG;
+  if (!aligned16(W_e4m3) || !aligned16(W_tiled)) return FP8BS_ERR_ALIGNMENT;
+  fp8bs_status st = check_device();
+  if (st != FP8BS_OK) return st;
+  return from_cuda(launch_tile_weight(W_e4m3, N, K, W_tiled, stream));
 }
 
 FP8BS_API fp8bs_status fp8bs_gemm_a8w8_blockscale(const void* A_e4m3, const float* a_scale, const void* W_e4m3,

@@ -87,6 +87,7 @@ struct F8Params {
   unsigned* counter;     // splits > 1: [tiles] arrival counters (left at zero)
   uint32_t wait_ns;            // bound of every wait (ns, below 2^32)
   int skip_it;                 // testing: CTA 0's producer skips this K-group iteration (-1: never)
+  const uint8_t* wt;           // tiled weights (16 KiB tiles, see tile_weight_kernel), or null
 };
 
 __device__ __forceinline__ uint32_t f8_timer() {  // low word of %globaltimer (ns; wraps every 4.3 s)
@@ -343,7 +344,14 @@ __global__ void __launch_bounds__(kF8Threads, 1)
           const uint32_t a_dst = smem_u32(smem + size_t(s) * C::kStageBytes);
           mbar_arrive_expect_tx(full_bar(s), C::kStageBytes);
           tma_load_2d(a_dst, &tmA, full_bar(s), kb * 128, tm * kF8BM);
-          tma_load_2d(a_dst + C::kABytes, &tmB, full_bar(s), kb * 128, tn * BN);
+          if (p.wt) {  // tiled weights: the BN / 128 tiles of this K group, each one contiguous copy
+#pragma unroll
+            for (int h = 0; h < BN / 128; ++h)
+              bulk_load(a_dst + C::kABytes + 16384 * h,
+                        p.wt + ((int64_t(tn) * (BN / 128) + h) * p.G + kb) * 16384, 16384, full_bar(s));
+          } else {
+            tma_load_2d(a_dst + C::kABytes, &tmB, full_bar(s), kb * 128, tn * BN);
+          }
         }
       }
       // drain (bounded, regardless of abort): the last issue of every stage has landed.
@@ -771,8 +779,11 @@ static int launch_f8(const void* A, const void* W, const F8Params& prm, void* st
     return e;
   CUtensorMap ma, mb, mo;
   if (!make_tma_2d_kmajor(&ma, A, true, prm.M, int64_t(prm.G) * 128, kF8BM) ||
-      !make_tma_2d_kmajor(&mb, W, true, prm.N, int64_t(prm.G) * 128, BN) ||
       !make_tma_2d_bf16_store(&mo, prm.out, prm.M, prm.N))
+    return int(cudaErrorInvalidValue);
+  if (prm.wt)
+    mb = ma;  // (unused: the weight tiles are plain copies)
+  else if (!make_tma_2d_kmajor(&mb, W, true, prm.N, int64_t(prm.G) * 128, BN))
     return int(cudaErrorInvalidValue);
   const int items = prm.m_tiles * prm.n_tiles * prm.splits;
   const int grid = std::min(items, device_sm_count());
@@ -881,7 +892,7 @@ size_t fp8_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, const KernelConfi
 }
 
 int launch_fp8_tc(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W, const float* w_scale,
-                  void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream) {
+                  void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream, bool tiled_w) {
   // the kernel indexes the scale matrices with 32-bit integers
   if (M * (K / 128) >= (int64_t(1) << 31) || ((N + 127) / 128) * (K / 128) >= (int64_t(1) << 31))
     return int(cudaErrorInvalidValue);
@@ -897,6 +908,7 @@ int launch_fp8_tc(const KernelConfig& cfg, const void* A, const float* a_scale, 
   p.splits = f8_splits(cfg, M, N, K);
   p.wait_ns = g_f8_wait_ns.load();
   p.skip_it = g_f8_skip_it.load();
+  p.wt = tiled_w ? static_cast<const uint8_t*>(W) : nullptr;
   if (p.splits > 1) {
     if (!ws) return int(cudaErrorInvalidValue);
     p.counter = static_cast<unsigned*>(ws);

@@ -111,6 +111,7 @@ struct GuParams {
   float* part;           // [2 * n_ctas][kGuSlots][kGuRows]
   unsigned* counter;     // [nblk]
   int out_fp32;          // bf16 GEMM only
+  const uint8_t* wt;     // tiled weights (16 KiB tiles, see tile_weight_kernel), or null
 };
 
 __device__ __forceinline__ void gu_put(const GuParams& p, int64_t idx, float v) {
@@ -306,7 +307,10 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
         for (int j = 0; j < pre; ++j) {
           const uint32_t dst = smem_u32(smem + size_t(j) * kGuStageBytes);
           mbar_arrive_expect_tx(full_bar(j), kTx);
-          tma_load_2d_hint(dst, &tmW, full_bar(j), pg * kX, pb * kGuRows, w_policy);
+          if (p.wt)  // tiled weights: the unit is one contiguous 16 KiB tile
+            bulk_load_hint(dst, p.wt + (int64_t(pb) * G + pg) * 16384, 16384, full_bar(j), w_policy);
+          else
+            tma_load_2d_hint(dst, &tmW, full_bar(j), pg * kX, pb * kGuRows, w_policy);
           if (++pg == G) {
             pg = 0;
             ++pb;
@@ -330,7 +334,10 @@ __global__ void __launch_bounds__(kGuThreads, kGuCtasPerSm)
         if (!mbar_wait_bounded(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, &g_status)) break;
         const uint32_t dst = smem_u32(smem + size_t(s) * kGuStageBytes);
         mbar_arrive_expect_tx(full_bar(s), kTx);
-        tma_load_2d_hint(dst, &tmW, full_bar(s), g * kX, b * kGuRows, w_policy);
+        if (p.wt)
+          bulk_load_hint(dst, p.wt + (int64_t(b) * G + g) * 16384, 16384, full_bar(s), w_policy);
+        else
+          tma_load_2d_hint(dst, &tmW, full_bar(s), g * kX, b * kGuRows, w_policy);
         tma_load_2d(dst + kGuWBytes, &tmA, full_bar(s), g * kX, 0);
         last_it[s] = it;
         if (++g == G) {
@@ -571,7 +578,7 @@ size_t gemv_umma_bf16_workspace_bytes(int64_t, int64_t N, int64_t K) { return gu
 
 template <int NT, bool kBf16>
 static int launch_gu(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out, int64_t M,
-                     int64_t N, int64_t K, void* ws, int static_w, int out_fp32, void* stream) {
+                     int64_t N, int64_t K, void* ws, int static_w, int out_fp32, void* stream, bool tiled_w = false) {
   // the carveout is a hint; the dynamic shared-memory limit is required (per device)
   if (const int attr = set_max_dynamic_smem(reinterpret_cast<const void*>(gemv_umma_kernel<NT, kBf16>),
                                             int(kGuSmemBytes)))
@@ -582,7 +589,10 @@ static int launch_gu(const void* A, const float* a_scale, const void* W, const f
                                int(cudaSharedmemCarveoutMaxShared));
   });
   CUtensorMap mw, ma;
-  if (!make_tma_2d_kmajor(&mw, W, !kBf16, N, K, kGuRows) || !make_tma_2d_kmajor(&ma, A, !kBf16, M, K, NT))
+  if (!make_tma_2d_kmajor(&ma, A, !kBf16, M, K, NT)) return int(cudaErrorInvalidValue);
+  if (tiled_w)
+    mw = ma;  // (unused: the weight tiles are plain copies)
+  else if (!make_tma_2d_kmajor(&mw, W, !kBf16, N, K, kGuRows))
     return int(cudaErrorInvalidValue);
   GuParams p{};
   p.a_scale = a_scale;
@@ -597,18 +607,23 @@ static int launch_gu(const void* A, const float* a_scale, const void* W, const f
   p.out_fp32 = kBf16 ? out_fp32 : 0;
   p.counter = static_cast<unsigned*>(ws);
   p.part = reinterpret_cast<float*>(static_cast<char*>(ws) + kCounterBytes);
+  p.wt = tiled_w ? static_cast<const uint8_t*>(W) : nullptr;
   return launch_kernel(gemv_umma_kernel<NT, kBf16>, dim3(p.n_ctas), dim3(kGuThreads), kGuSmemBytes, stream, mw, ma, p);
 }
 
 int launch_gemv_umma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
-                          int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream) {
+                          int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream, bool tiled_w) {
   if (M < 1 || M > kGemvMaxM || (N + kGuRows - 1) / kGuRows > kMaxCounters) return int(cudaErrorInvalidValue);
-  if (!gu_scales_fit(M, N, K))
+  if (!gu_scales_fit(M, N, K)) {
+    if (tiled_w) return int(cudaErrorNotSupported);  // (the mma.sync kernel reads the standard layout only)
     return launch_gemv_tma_a8w8(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, stream);
-  if (M <= 8) return launch_gu<8, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, 0, stream);
-  if (M <= 16) return launch_gu<16, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, 0, stream);
-  return launch_gu<32, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, 0, stream);
+  }
+  if (M <= 8) return launch_gu<8, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, 0, stream, tiled_w);
+  if (M <= 16) return launch_gu<16, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, 0, stream, tiled_w);
+  return launch_gu<32, false>(A, a_scale, W, w_scale, out, M, N, K, ws, static_w, 0, stream, tiled_w);
 }
+
+bool gemv_umma_reads_tiles(int64_t M, int64_t N, int64_t K) { return M >= 1 && M <= kGemvMaxM && gu_scales_fit(M, N, K); }
 
 int launch_gemv_umma_bf16(const void* A, const void* W, void* out, int out_fp32, int64_t M, int64_t N, int64_t K,
                           void* ws, void* stream) {

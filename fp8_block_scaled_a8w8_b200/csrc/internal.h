@@ -85,7 +85,13 @@ int launch_gemv_tma_a8w8(const void* A, const float* a_scale, const void* W, con
 
 size_t gemv_umma_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int launch_gemv_umma_a8w8(const void* A, const float* a_scale, const void* W, const float* w_scale, void* out,
-                          int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream);
+                          int64_t M, int64_t N, int64_t K, void* ws, int static_w, void* stream, bool tiled_w = false);
+// The decode kernel can read this shape's weights in the tiled layout (its scales fit the
+// staging region; otherwise the shape goes to the mma.sync kernel, which cannot).
+bool gemv_umma_reads_tiles(int64_t M, int64_t N, int64_t K);
+// Tiled weight layout: bytes of the tiles of an [N, K] e4m3 weight, and the tiling launch.
+size_t tiled_weight_bytes(int64_t N, int64_t K);
+int launch_tile_weight(const void* w, int64_t N, int64_t K, void* wt, void* stream);
 size_t gemv_umma_bf16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int launch_gemv_umma_bf16(const void* A, const void* W, void* out, int out_fp32, int64_t M, int64_t N, int64_t K,
                           void* ws, void* stream);
@@ -106,7 +112,8 @@ bool make_tma_2d_bf16_store(CUtensorMap* m, void* ptr, int64_t rows, int64_t col
 
 size_t fp8_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, const KernelConfig& cfg);
 int launch_fp8_tc(const KernelConfig& cfg, const void* A, const float* a_scale, const void* W, const float* w_scale,
-                  void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream);
+                  void* out, int64_t M, int64_t N, int64_t K, void* ws, void* stream,
+                  bool tiled_w = false);
 // MX32 GEMM (E8M0 scales on 32-wide K groups, hardware block scaling), batch >= 1.
 size_t mx_workspace_bytes(int64_t batch, int64_t M, int64_t N, int64_t K);
 int launch_gemm_mx32(const void* A, const uint8_t* a_e, const void* W, const uint8_t* w_e, void* out, int64_t batch,

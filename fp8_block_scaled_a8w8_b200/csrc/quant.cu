@@ -344,3 +344,46 @@ int launch_quant_weight(const float* w, int64_t N, int64_t K, void* q, float* sc
 }
 
 }  // namespace fp8bs
+
+namespace fp8bs {
+
+// ---------------------------------------------------------------- tiled weight layout
+// The e4m3 weight [N, K] rearranged into 16 KiB tiles, one per (128-row block b, 128-wide
+// K group g), tile (b, g) at byte (b * G + g) * 16384; inside a tile row r's 128 bytes sit
+// in the 128-byte-swizzled order the tensor core's K-major shared-memory operand uses
+// (16-byte chunk c of row r at chunk c ^ (r % 8)). So a tile is one contiguous copy that
+// lands in shared memory ready for the MMA -- the role of the pages' pre-shuffled B
+// ("bpreshuffle", [aiter#7247]), for this hardware. Rows past N and the padding block that
+// makes the block count even are zero. One CTA per tile, 256 threads, 4 x 16 bytes each.
+__global__ void __launch_bounds__(256) tile_weight_kernel(const uint8_t* __restrict__ w, int64_t N, int64_t K,
+                                                          uint8_t* __restrict__ wt) {
+  pdl_trigger();
+  pdl_wait();
+  const int64_t G = K / 128;
+  const int64_t tile = blockIdx.x;
+  const int64_t b = tile / G, g = tile - b * G;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int ci = threadIdx.x + 256 * k;  // destination 16-byte chunk of the tile
+    const int r = ci >> 3, c = (ci & 7) ^ (r & 7);
+    const int64_t row = b * 128 + r;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (row < N) v = ld_nc_v4(w + row * K + g * 128 + c * 16);
+    *reinterpret_cast<uint4*>(wt + tile * 16384 + ci * 16) = v;
+  }
+}
+
+size_t tiled_weight_bytes(int64_t N, int64_t K) {
+  const int64_t nblk = (N + 127) / 128;
+  return size_t((nblk + 1) / 2 * 2) * size_t(K / 128) * 16384;
+}
+
+int launch_tile_weight(const void* w, int64_t N, int64_t K, void* wt, void* stream) {
+  const int64_t nblk_pad = ((N + 127) / 128 + 1) & ~int64_t(1);
+  const int64_t tiles = nblk_pad * (K / 128);
+  if (tiles >= (int64_t(1) << 31)) return int(cudaErrorInvalidValue);
+  return launch_kernel(tile_weight_kernel, dim3(unsigned(tiles)), dim3(256), 0, stream,
+                       static_cast<const uint8_t*>(w), N, K, static_cast<uint8_t*>(wt));
+}
+
+}  // namespace fp8bs

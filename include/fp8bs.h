@@ -147,7 +147,12 @@ enum {
    * kernel then starts fetching W before the preceding kernel in the stream has finished
    * (programmatic dependent launch), overlapping its weight stream with that kernel's
    * tail; activations, scales and the workspace are still read only after it finished. */
-  FP8BS_FLAG_STATIC_WEIGHTS = 1u
+  FP8BS_FLAG_STATIC_WEIGHTS = 1u,
+  /* W_e4m3 points to the tiled layout written by fp8bs_tile_weight_e4m3 (not [N, K]).
+   * The call then runs the tcgen05 weight-streaming kernel (M <= 32) or the wide-epilogue
+   * tensor-core kernel (M > 32), whatever a table row names; a decode shape whose scales
+   * do not fit that kernel's staging area returns FP8BS_ERR_UNSUPPORTED. */
+  FP8BS_FLAG_TILED_WEIGHTS = 2u
 };
 
 /* fp8bs_gemm_a8w8_blockscale with flags (a bitwise OR of FP8BS_FLAG_*; unknown bits give
@@ -156,6 +161,21 @@ fp8bs_status fp8bs_gemm_a8w8_blockscale_ex(const void* A_e4m3, const float* a_sc
                                            const float* w_scale, void* out_bf16, int64_t M, int64_t N,
                                            int64_t K, void* workspace, size_t workspace_bytes, uint32_t flags,
                                            fp8bs_stream_t stream);
+
+/*
+ * Tiled weight layout (the role of the pages' pre-shuffled B, "bpreshuffle" [aiter#7247],
+ * for this hardware): W_e4m3 [N, K] rearranged into 16 KiB tiles, one per 128-row block b
+ * and 128-wide K group g, tile (b, g) at byte offset (b * K/128 + g) * 16384; within a tile,
+ * row r's 128 bytes in the order of the tensor core's 128-byte-swizzled K-major operand
+ * (16-byte chunk c stored at position c ^ (r % 8)). The block count is rounded up to an even
+ * number; rows past N are zero. Each tile is one contiguous copy into shared memory, which
+ * streams from HBM faster than the 128-byte row pieces of the [N, K] layout.
+ * fp8bs_tiled_weight_bytes: size of the tiled copy (0 for invalid sizes). Host only.
+ * fp8bs_tile_weight_e4m3: writes it (device pointers, both 16-byte aligned; K % 128 == 0);
+ * w_scale is unchanged. Pass the result with FP8BS_FLAG_TILED_WEIGHTS.
+ */
+size_t fp8bs_tiled_weight_bytes(int64_t N, int64_t K);
+fp8bs_status fp8bs_tile_weight_e4m3(const void* W_e4m3, int64_t N, int64_t K, void* W_tiled, fp8bs_stream_t stream);
 
 /*
  * The a8w8 block-scaled GEMM for decode-sized M without any caller-provided memory.
@@ -228,7 +248,9 @@ fp8bs_status fp8bs_gemm_bf16(const void* A_bf16, const void* W_bf16, void* out, 
                              int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                              fp8bs_stream_t stream);
 
-/* Bytes of workspace a call of op with this shape needs (0 if none). Host only. */
+/* Bytes of workspace a call of op with this shape needs (0 if none): enough for the
+ * configuration the dispatch table picks and for the shape's default configuration (which
+ * a call with FP8BS_FLAG_TILED_WEIGHTS may run instead). Host only. */
 size_t fp8bs_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
 /*
