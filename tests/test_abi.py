@@ -58,6 +58,14 @@ def test_argument_validation_without_gpu():
     # misaligned pointer
     assert l.fp8bs_gemm_a8w8_blockscale(P + 1, P, P, P, P, 1, 128, 128, None, 0, None) == 3
     assert l.fp8bs_gemm_bf16(P, P + 8, P, 0, 4, 32, 64, None, 0, None) == 3
+    # tiled weights: sizes, tiling arguments, unknown GEMM flag bits
+    assert fb.tiled_weight_bytes(5120, 6144) == 40 * 48 * 16384
+    assert fb.tiled_weight_bytes(400, 1408) == 4 * 11 * 16384  # block count rounded up to even
+    assert fb.tiled_weight_bytes(128, 100) == 0
+    assert l.fp8bs_tile_weight_e4m3(None, 128, 128, P, None) == 1
+    assert l.fp8bs_tile_weight_e4m3(P, 128, 100, P, None) == 1
+    assert l.fp8bs_tile_weight_e4m3(P, 128, 128, P + 4, None) == 3
+    assert l.fp8bs_gemm_a8w8_blockscale_ex(P, P, P, P, P, 1, 128, 128, None, 0, 4, None) == 1
     assert l.fp8bs_gemm_bf16(P, P, P, 0, 4, 32, 96, None, 0, None) == 1
     # quantisers: group must be 128, ld_x >= K and a multiple of 8
     assert l.fp8bs_quant_act_per_token_group(P, 2, 256, 256, P, P, 64, None) == 1
