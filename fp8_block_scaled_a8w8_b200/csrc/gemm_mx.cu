@@ -49,7 +49,7 @@ constexpr int kMxOutBytes = kMxEpiWarps * 2048;  // one 32 x 32 bf16 staging box
 // 8 weight-block words per stage, kMxSfAhead stages in flight
 constexpr int kMxSfSlotBytes = 512 + 32;
 constexpr int kMxSfRing = 8, kMxSfAhead = 6;
-constexpr int kMxSfBytes = 4 * kMxSfRing * kMxSfSlotBytes;
+constexpr int kMxSfBytes = kMxSfRing * kMxSfSlotBytes;
 constexpr size_t kMxSmemBytes = size_t(kMxStages) * kMxStageBytes + kMxOutBytes + kMxSfBytes + 1024 + 256;
 constexpr uint32_t kMxSfBase = 2 * kMxBN;  // TMEM: [2 accumulators][scale-factor slots of 32 columns]
 static_assert(kMxSfBase + 32 * kMxStages <= 512, "TMEM budget");
@@ -145,6 +145,21 @@ __device__ __forceinline__ uint32_t mx_pack_bf16x2(float a, float b) {
 }
 
 __device__ __forceinline__ void mx_epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// Barrier of the four scale-factor writer warps that also ANDs a flag over their threads,
+// so that all four leave their loop together (a warp that left alone would strand the
+// others at the next barrier).
+__device__ __forceinline__ bool mx_sf_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 3, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(v))
+      : "memory");
+  return r != 0;
+}
 
 // item -> (split, tile); tile -> (tm fastest, tn, batch)
 struct MxItem {
@@ -300,13 +315,14 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ scale-factor writers
     // Warp q writes TMEM lanes 32q..32q+31 (every subpartition holds the same copy). The
-    // scale bytes come from global memory (L2) with a latency of several stages, so each
-    // warp copies them kMxSfAhead stages ahead with cp.async into its own shared-memory
-    // ring: its lanes' 4 activation rows (4 bytes = 4 K groups each) and the tile's 6
-    // weight blocks, one commit group per stage.
+    // scale bytes come from global memory (L2) with a latency of several stages, so the
+    // four warps copy them kMxSfAhead stages ahead with cp.async into one shared-memory
+    // ring: per stage warp q fetches activation rows 32q .. 32q+31 (4 bytes = 4 K groups
+    // each) and warp 4 the tile's 6 weight blocks, one commit group per stage; a barrier of
+    // the four warps then makes every row visible to all of them.
     const int q = warp & 3;
     const uint32_t lane_addr = tmem_base + (uint32_t(32 * q) << 16);
-    const uint32_t ring = smem_u32(sf_ring + q * kMxSfRing * kMxSfSlotBytes);
+    const uint32_t ring = smem_u32(sf_ring);
     MxStageIter use_it(p, items), fetch_it(p, items);
     auto fetch = [&](int slot) {
       if (fetch_it.valid) {
@@ -314,14 +330,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         const uint8_t* arow = p.a_e + (int64_t(w.bt) * p.M) * p.K32 + 4 * fetch_it.kb;
         const uint8_t* wrow = p.w_e + (int64_t(w.bt) * p.NB32) * p.K32 + 4 * fetch_it.kb;
         const uint32_t base = ring + slot * kMxSfSlotBytes;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int r = min(w.tm * kMxBM + lane + 32 * j, p.M - 1);  // rows past M: any valid row
-          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + 4 * (32 * j + lane)),
-                       "l"(arow + int64_t(r) * p.K32)
-                       : "memory");
-        }
-        if (lane < kMxBN / 32) {
+        const int r = min(w.tm * kMxBM + 32 * q + lane, p.M - 1);  // rows past M: any valid row
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + 4 * (32 * q + lane)),
+                     "l"(arow + int64_t(r) * p.K32)
+                     : "memory");
+        if (q == 0 && lane < kMxBN / 32) {
           const int nb = min(w.tn * (kMxBN / 32) + lane, p.NB32 - 1);
           asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + 512 + 4 * lane),
                        "l"(wrow + int64_t(nb) * p.K32)
@@ -336,9 +349,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     int it = 0;
     for (; use_it.valid; ++it) {
       fetch((it + kMxSfAhead) % kMxSfRing);
-      asm volatile("cp.async.wait_group %0;" ::"n"(kMxSfAhead) : "memory");  // stage it's bytes have landed
-      __syncwarp();
+      asm volatile("cp.async.wait_group %0;" ::"n"(kMxSfAhead) : "memory");  // this warp's bytes of stage it
       const int s = it % S;
+      const bool ok = __all_sync(0xffffffffu, mx_wait(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, lim));
+      if (!mx_sf_bar_and(ok)) break;  // the other three warps' bytes too (the ring slot is complete)
       const uint32_t base = ring + (it % kMxSfRing) * kMxSfSlotBytes;
       uint32_t sa[4], sb[8];
 #pragma unroll
@@ -348,7 +362,6 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         sb[j] = 0x7F7F7F7Fu;
         if (j < kMxBN / 32) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sb[j]) : "r"(base + 512 + 4 * j));
       }
-      if (!__all_sync(0xffffffffu, mx_wait(empty_bar(s), ((it / S) & 1) ^ 1, abort_flag, lim))) break;
       tc_fence_after();
       const uint32_t slot = lane_addr + kMxSfBase + uint32_t(32 * s);
       mx_tmem_st_x4(slot, sa[0], sa[1], sa[2], sa[3]);  // column j: rows 32j + lane
