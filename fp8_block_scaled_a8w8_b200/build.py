@@ -46,7 +46,7 @@ REGISTER_CONTRACTS = {"gemm_tc.cu": ("gemm_tc_kernel", 168), "gemm_fp8.cu": ("ge
 # staged scales. The split-K tensor-core instantiations and rare fallbacks may spill a few
 # bytes and are not listed.
 SPILL_FREE = {"gemv_umma.cu": [r"gemv_umma_kernel"], "gemm_tc.cu": [r"gemm_tc_kernel.*Lb0EEEv"],
-              "gemv_tma.cu": [r"gemv_tma_kernel.*Lb1EEEv"], "gemm_fp8.cu": [r"gemm_fp8_kernel"], "gemm_mx.cu": [r"gemm_mx_kernel"]}
+              "gemv_tma.cu": [r"gemv_tma_kernel.*Lb1EEEv"], "gemm_fp8.cu": [r"gemm_fp8_kernel.*Lb0EEEv"], "gemm_mx.cu": [r"gemm_mx_kernel"]}
 
 
 def _check_spill_free(src: str, log: str) -> None:

@@ -39,6 +39,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "splitk.cuh"
 
 namespace fp8bs {
 
@@ -170,20 +171,6 @@ __device__ __forceinline__ uint32_t f8_pack_bf16x2(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// kCols consecutive columns of one output row as bf16, masked at M and N (N % 16 == 0,
-// so an 8-column chunk is either wholly inside or wholly outside).
-template <int kCols>
-__device__ __forceinline__ void f8_store_row(const F8Params& p, int row, int col, const float* v) {
-  if (row >= p.M) return;
-  __nv_bfloat16* dst = p.out + int64_t(row) * p.N + col;
-#pragma unroll
-  for (int j = 0; j < kCols; j += 8)
-    if (col + j < p.N)
-      *reinterpret_cast<uint4*>(dst + j) = make_uint4(f8_pack_bf16x2(v[j], v[j + 1]), f8_pack_bf16x2(v[j + 2], v[j + 3]),
-                                                      f8_pack_bf16x2(v[j + 4], v[j + 5]),
-                                                      f8_pack_bf16x2(v[j + 6], v[j + 7]));
-}
-
 // Output staging: each epilogue warp owns kF8OutBytesPerWarp of shared memory (32 rows x
 // 32 bf16, the 64-byte-swizzled layout of a 32 x 32 TMA store box).
 
@@ -221,48 +208,38 @@ __device__ __forceinline__ void f8_store_tile_tma(const CUtensorMap* tm_out, uin
   }
 }
 
-// Split K: publish this split's partial tile, and if it is the last split of the tile to
-// arrive, sum the tile's partials in split order, round once and reset the counter.
-// Every epilogue thread calls this for every item (also after an abort), so the
-// epilogue barriers always see all 512 threads.
+// Split K: store this split's partial tile, then finish the tile (splitk.cuh: the
+// distributed sum when every CTA holds one item, else the last split to arrive sums it).
+// Every epilogue thread calls this for every item (also after an abort), so the epilogue
+// barriers always see all 512 threads.
 template <int BN, int kCols>
 __device__ __forceinline__ void f8_splitk(const F8Params& p, int item, int tile, int row_in_tile, int row, int col0,
-                                          int cq, const float* acc, bool have, volatile unsigned* s_old,
-                                          volatile int* abort_flag) {
+                                          int cq, const float* acc, bool have, volatile int* flag,
+                                          volatile int* abort_flag, int items) {
   if (have && row < p.M) {
     float* dst = p.part + (int64_t(item) * kF8BM + row_in_tile) * BN + cq * kCols;
 #pragma unroll
     for (int j = 0; j < kCols; j += 4)
       __stcg(reinterpret_cast<float4*>(dst + j), make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]));
   }
-  f8_epilogue_bar();  // every epilogue thread's partial stores precede the release below
+  const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
+  const int row0 = tm * kF8BM, tcol0 = tn * BN;
+  SplitTile t;
+  t.part = p.part + int64_t(tile) * p.splits * kF8BM * BN;
+  t.split_elems = kF8BM * BN;
+  t.ld = BN;
+  t.rows = min(kF8BM, p.M - row0);
+  t.qpr = min(BN, p.N - tcol0) / 4;
+  __nv_bfloat16* const out_t = p.out + int64_t(row0) * p.N + tcol0;
+  const int ldo = p.N;
+  auto store = [out_t, ldo](int r, int c, float4 s) {
+    *reinterpret_cast<uint2*>(out_t + int64_t(r) * ldo + c) =
+        make_uint2(f8_pack_bf16x2(s.x, s.y), f8_pack_bf16x2(s.z, s.w));
+  };
   // after a timed-out wait nothing is published (the status word reports it; the caller
   // re-zeroes the workspace before reusing it)
-  if (threadIdx.x == 128) *s_old = *abort_flag ? ~0u : atom_add_acq_rel_gpu(p.counter + tile, 1u);
-  f8_epilogue_bar();
-  if (*s_old != unsigned(p.splits - 1)) return;
-  if (row < p.M) {
-#pragma unroll 1
-    for (int c = 0; c < kCols; c += 32) {
-      float sum[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) sum[j] = 0.f;
-#pragma unroll 1
-      for (int sp = 0; sp < p.splits; ++sp) {
-        const float* src = p.part + ((int64_t(tile) * p.splits + sp) * kF8BM + row_in_tile) * BN + cq * kCols + c;
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          const float4 f = __ldcg(reinterpret_cast<const float4*>(src + j));
-          sum[j] += f.x;
-          sum[j + 1] += f.y;
-          sum[j + 2] += f.z;
-          sum[j + 3] += f.w;
-        }
-      }
-      f8_store_row<32>(p, row, col0 + c, sum);
-    }
-  }
-  if (threadIdx.x == 128) p.counter[tile] = 0u;
+  splitk_finish(p.counter + tile, t, p.splits, item - tile * p.splits, have && !*abort_flag, items,
+                int(threadIdx.x) - 128, kF8EpiThreads, flag, p.wait_ns, &g_status, f8_epilogue_bar, store);
 }
 
 template <int BN, bool kSplitK>
@@ -283,7 +260,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
   uint32_t* tmem_slot = misc;
   const uint32_t abort_addr = smem_u32(misc + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-  volatile unsigned* s_old = reinterpret_cast<volatile unsigned*>(misc + 2);
+  volatile int* split_flag = reinterpret_cast<volatile int*>(misc + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -455,7 +432,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
         f8_store_tile_tma<kCols>(&tmOut, smem_u32(out_stage + (warp - 4) * kF8OutBytesPerWarp), tm * kF8BM + 32 * q,
                                  col0, acc);
       } else {
-        f8_splitk<BN, kCols>(p, item, tile, row_in_tile, row, col0, cq, acc, ok, s_old, abort_flag);
+        f8_splitk<BN, kCols>(p, item, tile, row_in_tile, row, col0, cq, acc, ok, split_flag, abort_flag, items);
       }
     }
   }

@@ -20,8 +20,8 @@
 //                 MMA's scale-factor operands)
 //   warps 8..15   epilogue: TMEM -> bf16 -> shared memory -> TMA store (two TMEM
 //                 accumulators alternate between tiles)
-// Small tile counts split K: each split stores the rows < M of its fp32 tile, the last to
-// arrive (gpu-scope acq_rel counter) sums them in split order and writes bf16.
+// Small tile counts split K: each split stores the rows < M of its fp32 tile and the tile
+// is finished as splitk.cuh describes (partials summed in split order, rounded once).
 // Every wait is bounded; on expiry the CTA raises its abort flag and the status word,
 // drains what it issued and frees TMEM.
 #include <cuda.h>
@@ -34,6 +34,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "splitk.cuh"
 
 namespace fp8bs {
 
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   uint32_t* misc = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
   uint32_t* tmem_slot = misc;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
-  volatile unsigned* s_old = reinterpret_cast<volatile unsigned*>(misc + 2);
+  volatile int* split_flag = reinterpret_cast<volatile int*>(misc + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -436,53 +437,21 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
       }
       if constexpr (kSplitK) {
-        // publish this split; the last split of the tile sums the partials in split order
-        mx_epi_bar();
-        if (threadIdx.x == 256) *s_old = (!ok || *abort_flag) ? ~0u : atom_add_acq_rel_gpu(p.counter + w.tile, 1u);
-        mx_epi_bar();
-        if (*s_old == unsigned(p.splits - 1)) {
-          const int row = row0 + lane;
-          if (row < p.M) {
-#pragma unroll 1
-            for (int c = 0; c < kMxBN / 64; ++c) {
-              float sum[32];
-#pragma unroll
-              for (int j = 0; j < 32; ++j) sum[j] = 0.f;
-#pragma unroll 1
-              for (int sp0 = 0; sp0 < p.splits; sp0 += 2) {  // two splits' loads in flight (16 x 16 B)
-                float4 f[2][8];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                  const int sp = sp0 + u < p.splits ? sp0 + u : sp0;
-                  const float* src = p.part + ((int64_t(w.tile) * p.splits + sp) * kMxBM + 32 * q + lane) * kMxBN +
-                                     h * (kMxBN / 2) + 32 * c;
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) f[u][j] = __ldcg(reinterpret_cast<const float4*>(src + 4 * j));
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                  if (sp0 + u >= p.splits) break;
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) {
-                    sum[4 * j] += f[u][j].x;
-                    sum[4 * j + 1] += f[u][j].y;
-                    sum[4 * j + 2] += f[u][j].z;
-                    sum[4 * j + 3] += f[u][j].w;
-                  }
-                }
-              }
-              const int col0 = col_base + 32 * c;
-              __nv_bfloat16* dst = p.out + (int64_t(w.bt) * p.M + row) * p.N + col0;
-#pragma unroll
-              for (int j = 0; j < 32; j += 8)
-                if (col0 + j < p.N)
-                  *reinterpret_cast<uint4*>(dst + j) =
-                      make_uint4(mx_pack_bf16x2(sum[j], sum[j + 1]), mx_pack_bf16x2(sum[j + 2], sum[j + 3]),
-                                 mx_pack_bf16x2(sum[j + 4], sum[j + 5]), mx_pack_bf16x2(sum[j + 6], sum[j + 7]));
-            }
-          }
-          if (threadIdx.x == 256) p.counter[w.tile] = 0u;
-        }
+        // publish this split and finish the tile (splitk.cuh): the partials in split order
+        const int trow0 = w.tm * kMxBM, tcol0 = w.tn * kMxBN;
+        SplitTile t;
+        t.part = p.part + int64_t(w.tile) * p.splits * kMxBM * kMxBN;
+        t.split_elems = kMxBM * kMxBN;
+        t.ld = kMxBN;
+        t.rows = min(kMxBM, p.M - trow0);
+        t.qpr = min(kMxBN, p.N - tcol0) / 4;
+        __nv_bfloat16* out_t = p.out + (int64_t(w.bt) * p.M + trow0) * p.N + tcol0;
+        auto store = [&](int r, int c, float4 s) {
+          *reinterpret_cast<uint2*>(out_t + int64_t(r) * p.N + c) =
+              make_uint2(mx_pack_bf16x2(s.x, s.y), mx_pack_bf16x2(s.z, s.w));
+        };
+        splitk_finish(p.counter + w.tile, t, p.splits, w.sp, ok && !*abort_flag, items,
+                      int(threadIdx.x) - 256, 256, split_flag, lim, &g_status, mx_epi_bar, store);
       } else {
         if (!ok) break;
       }
@@ -523,9 +492,9 @@ static int mx_splits(int64_t batch, int64_t M, int64_t N, int64_t K) {
   const int64_t kb = K / 128;
   const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + kMxBN - 1) / kMxBN);
   const int64_t sms = device_sm_count();
-  // one wave (tiles x splits <= SMs), and at most 4 splits: one CTA sums a tile's partials
-  // (two splits' loads in flight), so each further split adds a round trip to the finish
-  int64_t sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({sms / tiles, kb / 2, 4});
+  // one wave (tiles x splits <= SMs), at most 8 splits (the finish loads every split of an
+  // element at once), each split at least 2 K blocks
+  int64_t sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({sms / tiles, kb / 2, 8});
   sp = std::max<int64_t>(1, std::min(sp, kb));
   if (sp > 1 && tiles > kMaxCounters) sp = 1;
   return int(sp);

@@ -28,6 +28,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "splitk.cuh"
 
 namespace fp8bs {
 
@@ -124,10 +125,9 @@ __device__ __forceinline__ void store_row_chunk(const TcParams& p, int row, int 
   }
 }
 
-// Split K: every split stores its float32 partial tile; after all epilogue threads have
-// stored, one thread counts the split in (gpu-scope acq_rel atomic after the epilogue
-// barrier), and the split that arrives last sums the tile's partials in split order -- a
-// fixed order, so results are bit-reproducible -- rounds once and resets the counter.
+// Split K: every split stores its float32 partial tile, then the tile is finished as
+// splitk.cuh describes (the distributed sum when every CTA holds one item, else the last
+// split to arrive sums it): the partials in split order, rounded once.
 template <int kChunk>
 __device__ __forceinline__ void tc_store_partial(const TcParams& p, float* dst, int row, const float* v) {
   if (row >= p.M) return;
@@ -135,46 +135,29 @@ __device__ __forceinline__ void tc_store_partial(const TcParams& p, float* dst, 
   for (int j = 0; j < kChunk; j += 4) __stcg(reinterpret_cast<float4*>(dst + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
 }
 
-template <int BN, int kHalf, int kChunk>
-__device__ __forceinline__ void tc_splitk_finish(const TcParams& p, int tile, int row_in_tile, int row, int h,
-                                                 int col0, volatile unsigned* s_old, volatile int* abort_flag) {
-  tc_epilogue_bar();  // every epilogue thread's partial stores precede the release below
+template <int BN>
+__device__ __forceinline__ void tc_splitk_finish(const TcParams& p, int item, int tile, volatile int* flag,
+                                                 volatile int* abort_flag, int items) {
+  const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
+  const int row0 = tm * kBM, tcol0 = tn * BN;
+  SplitTile t;
+  t.part = p.part + int64_t(tile) * p.splits * kBM * BN;
+  t.split_elems = kBM * BN;
+  t.ld = BN;
+  t.rows = min(kBM, p.M - row0);
+  t.qpr = min(BN, p.N - tcol0) / 4;
+  auto store = [&](int r, int c, float4 s) {
+    const int64_t o = int64_t(row0 + r) * p.N + tcol0 + c;
+    if (p.out_fp32)
+      *reinterpret_cast<float4*>(static_cast<float*>(p.out) + o) = s;
+    else
+      *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.out) + o) =
+          make_uint2(pack_bf16x2(s.x, s.y), pack_bf16x2(s.z, s.w));
+  };
   // after a timed-out wait nothing is published (the status word reports it; the caller
   // re-zeroes the workspace before reusing it)
-  if (threadIdx.x == 128) *s_old = *abort_flag ? ~0u : atom_add_acq_rel_gpu(p.counter + tile, 1u);
-  tc_epilogue_bar();
-  if (*s_old != unsigned(p.splits - 1)) return;
-  if (row < p.M) {
-#pragma unroll 1
-    for (int c = 0; c < kHalf / kChunk; ++c) {
-      float sum[kChunk];
-#pragma unroll
-      for (int j = 0; j < kChunk; ++j) sum[j] = 0.f;
-      constexpr int kPar = kChunk >= 32 ? 2 : 4;  // splits' loads in flight (64 floats)
-#pragma unroll 1
-      for (int sp = 0; sp < p.splits; sp += kPar) {
-        float v[kPar][kChunk];
-#pragma unroll
-        for (int k = 0; k < kPar; ++k) {
-          const float* src = p.part + ((int64_t(tile) * p.splits + sp + k) * kBM + row_in_tile) * BN + h * kHalf + c * kChunk;
-#pragma unroll
-          for (int j = 0; j < kChunk; j += 4) {
-            const float4 f = sp + k < p.splits ? __ldcg(reinterpret_cast<const float4*>(src + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
-            v[k][j] = f.x;
-            v[k][j + 1] = f.y;
-            v[k][j + 2] = f.z;
-            v[k][j + 3] = f.w;
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < kPar; ++k)
-#pragma unroll
-          for (int j = 0; j < kChunk; ++j) sum[j] += v[k][j];
-      }
-      store_row_chunk<kChunk>(p, row, col0 + c * kChunk, sum);
-    }
-  }
-  if (threadIdx.x == 128) p.counter[tile] = 0u;
+  splitk_finish(p.counter + tile, t, p.splits, item - tile * p.splits, !*abort_flag, items, int(threadIdx.x) - 128,
+                256, flag, kWaitLimitNs, &g_status, tc_epilogue_bar, store);
 }
 
 // kSplitK: instantiated with split-K support; without it the kernel is exactly the
@@ -192,7 +175,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // bars: full[S], empty[S], tmem_full[2], tmem_empty[2], drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile unsigned* s_old = reinterpret_cast<volatile unsigned*>(tmem_slot + 2);  // split-K arrival
+  volatile int* split_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);  // split-K finish
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -426,7 +409,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int c = 0; c < C::kChunks; ++c)
               tc_store_partial<C::kChunk>(p, part_row + c * C::kChunk, row, acc + c * C::kChunk);
           }
-          tc_splitk_finish<BN, C::kHalfCols, C::kChunk>(p, tile, row_in_tile, row, h, col0, s_old, abort_flag);
+          tc_splitk_finish<BN>(p, item, tile, split_flag, abort_flag, items);
         }
       } else {
         const int b = tile_it & 1;
@@ -454,7 +437,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(tempty_bar(b));
         }
-        if (kSplitK) tc_splitk_finish<BN, C::kHalfCols, C::kChunk>(p, tile, row_in_tile, row, h, col0, s_old, abort_flag);
+        if (kSplitK) tc_splitk_finish<BN>(p, item, tile, split_flag, abort_flag, items);
       }
     }
   }
