@@ -217,17 +217,18 @@ __device__ __forceinline__ void f8_splitk(const F8Params& p, int item, int tile,
                                           int cq, const float* acc, bool have, volatile int* flag,
                                           volatile int* abort_flag, int items) {
   if (have && row < p.M) {
-    float* dst = p.part + (int64_t(item) * kF8BM + row_in_tile) * BN + cq * kCols;
+    float* part_item = p.part + int64_t(item) * kF8BM * BN;
 #pragma unroll
     for (int j = 0; j < kCols; j += 4)
-      __stcg(reinterpret_cast<float4*>(dst + j), make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]));
+      __stcg(reinterpret_cast<float4*>(splitk_quad(part_item, kF8BM, row_in_tile, cq * kCols + j)),
+             make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]));
   }
   const int tm = tile % p.m_tiles, tn = tile / p.m_tiles;
   const int row0 = tm * kF8BM, tcol0 = tn * BN;
   SplitTile t;
   t.part = p.part + int64_t(tile) * p.splits * kF8BM * BN;
   t.split_elems = kF8BM * BN;
-  t.ld = BN;
+  t.bm = kF8BM;
   t.rows = min(kF8BM, p.M - row0);
   t.qpr = min(BN, p.N - tcol0) / 4;
   __nv_bfloat16* const out_t = p.out + int64_t(row0) * p.N + tcol0;
@@ -292,13 +293,14 @@ __global__ void __launch_bounds__(kF8Threads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_wait();  // the previous kernel's results are visible from here
+  // launch-time values before the grid-dependency wait (they do not depend on the
+  // previous kernel), so their first parameter reads overlap it
   const uint32_t tmem_base = *tmem_slot;
-
   const int splits = kSplitK ? p.splits : 1;
   const int items = p.m_tiles * p.n_tiles * splits;
   const int KB = p.G;
   const uint32_t lim = p.wait_ns;
+  pdl_wait();  // the previous kernel's results are visible from here
 
   if (warp < 4) {
     f8_setmaxnreg_dec<kF8ProducerRegs>();

@@ -250,11 +250,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_wait();
+  // launch-time values before the grid-dependency wait (they do not depend on the
+  // previous kernel), so their first parameter reads overlap it
   const uint32_t tmem_base = *tmem_slot;
   const int splits = kSplitK ? p.splits : 1;
   const int items = p.batch * p.m_tiles * p.n_tiles * splits;
   const uint32_t lim = p.wait_ns;
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -426,10 +428,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           } else {
             const int row = row0 + lane;
             if (row < p.M) {
-              float* dst = p.part + (int64_t(item) * kMxBM + 32 * q + lane) * kMxBN + h * (kMxBN / 2) + 32 * c;
+              float* part_item = p.part + int64_t(item) * kMxBM * kMxBN;
 #pragma unroll
               for (int j = 0; j < 32; j += 4)
-                __stcg(reinterpret_cast<float4*>(dst + j),
+                __stcg(reinterpret_cast<float4*>(splitk_quad(part_item, kMxBM, 32 * q + lane, h * (kMxBN / 2) + 32 * c + j)),
                        make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
                                    __uint_as_float(r[j + 3])));
             }
@@ -442,7 +444,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         SplitTile t;
         t.part = p.part + int64_t(w.tile) * p.splits * kMxBM * kMxBN;
         t.split_elems = kMxBM * kMxBN;
-        t.ld = kMxBN;
+        t.bm = kMxBM;
         t.rows = min(kMxBM, p.M - trow0);
         t.qpr = min(kMxBN, p.N - tcol0) / 4;
         __nv_bfloat16* out_t = p.out + (int64_t(w.bt) * p.M + trow0) * p.N + tcol0;

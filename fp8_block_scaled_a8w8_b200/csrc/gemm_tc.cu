@@ -128,11 +128,15 @@ __device__ __forceinline__ void store_row_chunk(const TcParams& p, int row, int 
 // Split K: every split stores its float32 partial tile, then the tile is finished as
 // splitk.cuh describes (the distributed sum when every CTA holds one item, else the last
 // split to arrive sums it): the partials in split order, rounded once.
-template <int kChunk>
-__device__ __forceinline__ void tc_store_partial(const TcParams& p, float* dst, int row, const float* v) {
+template <int BN, int kChunk>
+__device__ __forceinline__ void tc_store_partial(const TcParams& p, int item, int row_in_tile, int col, int row,
+                                                 const float* v) {
   if (row >= p.M) return;
+  float* part_item = p.part + int64_t(item) * kBM * BN;
 #pragma unroll
-  for (int j = 0; j < kChunk; j += 4) __stcg(reinterpret_cast<float4*>(dst + j), make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
+  for (int j = 0; j < kChunk; j += 4)
+    __stcg(reinterpret_cast<float4*>(splitk_quad(part_item, kBM, row_in_tile, col + j)),
+           make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]));
 }
 
 template <int BN>
@@ -143,7 +147,7 @@ __device__ __forceinline__ void tc_splitk_finish(const TcParams& p, int item, in
   SplitTile t;
   t.part = p.part + int64_t(tile) * p.splits * kBM * BN;
   t.split_elems = kBM * BN;
-  t.ld = BN;
+  t.bm = kBM;
   t.rows = min(kBM, p.M - row0);
   t.qpr = min(BN, p.N - tcol0) / 4;
   auto store = [&](int r, int c, float4 s) {
@@ -207,14 +211,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  pdl_wait();  // the previous kernel's results are visible from here
+  // launch-time values before the grid-dependency wait (they do not depend on the
+  // previous kernel), so their first parameter reads overlap it
   const uint32_t tmem_base = *tmem_slot;
-
   // work items: (output tile, K split); item -> tile = item / splits, K blocks [kb0, kb1)
   const int splits = kSplitK ? p.splits : 1;
   const int items = p.m_tiles * p.n_tiles * splits;
   const int KB = p.kblocks;
   const int G = p.K / 128;  // scale groups (a8w8)
+  pdl_wait();  // the previous kernel's results are visible from here
 
   if (warp < 4) {
    setmaxnreg_dec<kProducerRegs>();  // warpgroup 0 hands registers to the epilogue
@@ -404,10 +409,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int c = 0; c < C::kChunks; ++c) store_row_chunk<C::kChunk>(p, row, col0 + c * C::kChunk, acc + c * C::kChunk);
         } else {
           if (ok) {
-            float* part_row = p.part + (int64_t(item) * kBM + row_in_tile) * BN + h * C::kHalfCols;
 #pragma unroll
             for (int c = 0; c < C::kChunks; ++c)
-              tc_store_partial<C::kChunk>(p, part_row + c * C::kChunk, row, acc + c * C::kChunk);
+              tc_store_partial<BN, C::kChunk>(p, item, row_in_tile, h * C::kHalfCols + c * C::kChunk, row,
+                                              acc + c * C::kChunk);
           }
           tc_splitk_finish<BN>(p, item, tile, split_flag, abort_flag, items);
         }
@@ -430,8 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!kSplitK)
               store_row_chunk<C::kChunk>(p, row, col0 + c * C::kChunk, v);
             else
-              tc_store_partial<C::kChunk>(
-                  p, p.part + (int64_t(item) * kBM + row_in_tile) * BN + h * C::kHalfCols + c * C::kChunk, row, v);
+              tc_store_partial<BN, C::kChunk>(p, item, row_in_tile, h * C::kHalfCols + c * C::kChunk, row, v);
           }
           tc_fence_before();
           __syncwarp();
