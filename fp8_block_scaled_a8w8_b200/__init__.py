@@ -290,8 +290,14 @@ FLAG_STATIC_WEIGHTS = 1
 FLAG_TILED_WEIGHTS = 2
 
 
+_tiled_bytes = {}
+
+
 def tiled_weight_bytes(N: int, K: int) -> int:
-    return int(lib().fp8bs_tiled_weight_bytes(N, K))
+    v = _tiled_bytes.get((N, K))
+    if v is None:
+        v = _tiled_bytes[(N, K)] = int(lib().fp8bs_tiled_weight_bytes(N, K))
+    return v
 
 
 def tile_weight(W: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
@@ -331,9 +337,8 @@ def gemm_a8w8_blockscale(A: torch.Tensor, a_scale: torch.Tensor, W: torch.Tensor
             raise ValueError("operands must be contiguous")
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
-    need = workspace_bytes(OP_A8W8_BLOCKSCALE, M, N, K)
-    if workspace is None:
-        workspace = _workspace_for(A.device, need)
+    if workspace is None:  # a caller's workspace is size-checked by the C entry point
+        workspace = _workspace_for(A.device, workspace_bytes(OP_A8W8_BLOCKSCALE, M, N, K))
     ws_ptr = _ptr(workspace) if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
     flags = (FLAG_STATIC_WEIGHTS if static_weights else 0) | (FLAG_TILED_WEIGHTS if tiled_weights else 0)
@@ -372,9 +377,8 @@ def gemm_bf16(A: torch.Tensor, W: torch.Tensor, out_fp32: bool = False, out: tor
     N = W.shape[0]
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=A.device)
-    need = workspace_bytes(OP_BF16, M, N, K)
-    if workspace is None:
-        workspace = _workspace_for(A.device, need)
+    if workspace is None:  # a caller's workspace is size-checked by the C entry point
+        workspace = _workspace_for(A.device, workspace_bytes(OP_BF16, M, N, K))
     ws_ptr = _ptr(workspace) if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("fp8bs_gemm_bf16",
