@@ -48,7 +48,8 @@ def _check(x, r, g, res_out, q, s):
             assert abs(t - mid) <= 1e-5 * abs(t) + 1e-30, (m, k, t, a, b)
 
 
-@pytest.mark.parametrize("M,K", [(1, 128), (3, 384), (16, 5120), (130, 6144), (1000, 1024), (8, 8192)])
+@pytest.mark.parametrize("M,K", [(1, 128), (3, 384), (16, 5120), (130, 6144), (1000, 1024), (8, 8192), (300, 6144),
+                                 (257, 8192)])
 def test_add_rmsnorm_quant_parity(M, K):
     x, r, g = _inputs(M, K, M + K)
     res_out, q, s = fb.add_rmsnorm_quant(x.cuda(), r.cuda(), g.cuda(), EPS)
