@@ -48,8 +48,10 @@ def _a8w8(M, N, K, seed):
 @pytest.mark.parametrize("M,N,K,cfg,splits", [
     (48, 2048, 4096, "a8w8_tcw_bn256", 8),      # 8 tiles x 8 splits: distributed
     (100, 400, 1024, "a8w8_tcw_bn256", 4),      # ragged M and N tails, 2 tiles x 4 splits
+    (40, 256, 6144, "a8w8_tcw_bn256", 8),       # one tile, 8 splits
     (48, 5120, 6144, "a8w8_tc_bn128", 3),       # two-buffer kernel, 40 tiles x 3 splits
     (256, 2560, 2048, "a8w8_tcw_bn128_sk8", 8),  # 40 tiles x 8 = 320 items: last arrival
+    (256, 1024, 2048, "a8w8_tcw_bn128_sk8", 8),  # 16 tiles x 8 = 128 items: distributed
     (130, 1040, 1152, "a8w8_tcw_bn256_sk2", 2),  # 10 tiles x 2 splits, ragged tails
 ])
 def test_a8w8_split_finish(M, N, K, cfg, splits):
