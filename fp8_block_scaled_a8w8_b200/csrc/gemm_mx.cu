@@ -41,9 +41,9 @@ namespace fp8bs {
 FP8BS_DEFINE_STATUS(mx)
 
 constexpr int kMxThreads = 512;
-constexpr int kMxBM = 128, kMxBN = 192;
+constexpr int kMxBM = 128;
 constexpr int kMxStages = 4;
-constexpr int kMxABytes = kMxBM * 128, kMxBBytes = kMxBN * 128, kMxStageBytes = kMxABytes + kMxBBytes;
+constexpr int kMxABytes = kMxBM * 128;
 constexpr int kMxEpiWarps = 8;
 constexpr int kMxOutBytes = kMxEpiWarps * 2048;  // one 32 x 32 bf16 staging box per epilogue warp
 // scale-byte prefetch ring of each scale-factor writer warp: 128 activation-row words +
@@ -51,11 +51,21 @@ constexpr int kMxOutBytes = kMxEpiWarps * 2048;  // one 32 x 32 bf16 staging box
 constexpr int kMxSfSlotBytes = 512 + 32;
 constexpr int kMxSfRing = 8, kMxSfAhead = 6;
 constexpr int kMxSfBytes = kMxSfRing * kMxSfSlotBytes;
-constexpr size_t kMxSmemBytes = size_t(kMxStages) * kMxStageBytes + kMxOutBytes + kMxSfBytes + 1024 + 256;
-constexpr uint32_t kMxSfBase = 2 * kMxBN;  // TMEM: [2 accumulators][scale-factor slots of 32 columns]
-static_assert(kMxSfBase + 32 * kMxStages <= 512, "TMEM budget");
-static_assert(kMxStageBytes % 1024 == 0, "stage alignment");
-static_assert(kMxSmemBytes <= 232448, "shared memory per block");
+// Tile width BN: 192 with two TMEM accumulators alternating between tiles, or 256 with
+// one (for launches whose tiles fit one wave, where no CTA has a next tile to overlap).
+template <int BN>
+struct MxCfg {
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kStageBytes = kMxABytes + kBBytes;
+  static constexpr int kBufs = (2 * BN + 32 * kMxStages <= 512) ? 2 : 1;
+  static constexpr uint32_t kSfBase = uint32_t(kBufs * BN);  // TMEM: [accumulators][scale-factor slots, 32 columns]
+  static constexpr size_t kSmemBytes = size_t(kMxStages) * kStageBytes + kMxOutBytes + kMxSfBytes + 1024 + 256;
+  static_assert(BN == 192 || BN == 256, "tile width");
+  static_assert(kSfBase + 32 * kMxStages <= 512, "TMEM budget");
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+  static_assert(kSmemBytes <= 232448, "shared memory per block");
+  static_assert(BN / 32 <= 8, "weight-block scale words per stage");
+};
 
 struct MxParams {
   const uint8_t* a_e;   // [batch][M][K/32] E8M0
@@ -63,7 +73,7 @@ struct MxParams {
   __nv_bfloat16* out;   // [batch][M][N]
   int M, N, K32, KB, NB32, batch;
   int m_tiles, n_tiles, splits;
-  float* part;          // splits > 1: [items][kMxBM][kMxBN] float32 partial tiles
+  float* part;          // splits > 1: [items][kMxBM][BN] float32 partial tiles
   unsigned* counter;    // splits > 1: [tiles]
   uint32_t wait_ns;
 };
@@ -202,15 +212,17 @@ struct MxStageIter {
   }
 };
 
-template <bool kSplitK>
+template <bool kSplitK, int BN>
 __global__ void __launch_bounds__(kMxThreads, 1)
     gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmOut, const MxParams p) {
+  using C = MxCfg<BN>;
   constexpr int S = kMxStages;
+  constexpr int NB = C::kBufs;
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* out_stage = smem + size_t(S) * kMxStageBytes;
+  uint8_t* out_stage = smem + size_t(S) * C::kStageBytes;
   uint8_t* sf_ring = out_stage + kMxOutBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sf_ring + kMxSfBytes);
   // bars: full[S], empty[S], sf_full[S], tfull[2], tempty[2], drain
@@ -271,10 +283,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             ok = false;
             break;
           }
-          const uint32_t dst = smem_u32(smem + size_t(s) * kMxStageBytes);
-          mbar_arrive_expect_tx(full_bar(s), kMxStageBytes);
+          const uint32_t dst = smem_u32(smem + size_t(s) * C::kStageBytes);
+          mbar_arrive_expect_tx(full_bar(s), C::kStageBytes);
           mx_tma_load_3d(dst, &tmA, full_bar(s), kb * 128, w.tm * kMxBM, w.bt);
-          mx_tma_load_3d(dst + kMxABytes, &tmB, full_bar(s), kb * 128, w.tn * kMxBN, w.bt);
+          mx_tma_load_3d(dst + kMxABytes, &tmB, full_bar(s), kb * 128, w.tn * BN, w.bt);
         }
       }
       for (int j = it > S ? it - S : 0; j < it; ++j) mx_drain(full_bar(j % S), (j / S) & 1, lim);
@@ -286,10 +298,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       bool ok = true, issued = false;
       for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++tile_it) {
         const MxItem w = mx_item(p, item);
-        const int b = tile_it & 1;
-        if (!mx_wait(tempty_bar(b), ((tile_it >> 1) & 1) ^ 1, abort_flag, lim)) break;
+        const int b = tile_it % NB;
+        if (!mx_wait(tempty_bar(b), ((tile_it / NB) & 1) ^ 1, abort_flag, lim)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + uint32_t(b * kMxBN);
+        const uint32_t d_tmem = tmem_base + uint32_t(b * BN);
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const int s = it % S;
           if (!mx_wait(full_bar(s), (it / S) & 1, abort_flag, lim) ||
@@ -298,12 +310,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + size_t(s) * kMxStageBytes);
+          const uint32_t a_addr = smem_u32(smem + size_t(s) * C::kStageBytes);
           const uint64_t adesc = sw128_kmajor_desc(a_addr), bdesc = sw128_kmajor_desc(a_addr + kMxABytes);
-          const uint32_t sfa = tmem_base + kMxSfBase + uint32_t(32 * s), sfb = sfa + 16;
+          const uint32_t sfa = tmem_base + C::kSfBase + uint32_t(32 * s), sfb = sfa + 16;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mx_mma(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, mx_idesc(kMxBM, kMxBN, kk), sfa, sfb,
+            mx_mma(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, mx_idesc(kMxBM, BN, kk), sfa, sfb,
                    (kb > w.kb0 || kk > 0) ? 1u : 0u);
           issued = true;
           umma_commit(empty_bar(s));  // the stage and its scale-factor slot are free
@@ -337,8 +349,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + 4 * (32 * q + lane)),
                      "l"(arow + int64_t(r) * p.K32)
                      : "memory");
-        if (q == 0 && lane < kMxBN / 32) {
-          const int nb = min(w.tn * (kMxBN / 32) + lane, p.NB32 - 1);
+        if (q == 0 && lane < BN / 32) {
+          const int nb = min(w.tn * (BN / 32) + lane, p.NB32 - 1);
           asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + 512 + 4 * lane),
                        "l"(wrow + int64_t(nb) * p.K32)
                        : "memory");
@@ -363,10 +375,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         sb[j] = 0x7F7F7F7Fu;
-        if (j < kMxBN / 32) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sb[j]) : "r"(base + 512 + 4 * j));
+        if (j < BN / 32) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sb[j]) : "r"(base + 512 + 4 * j));
       }
       tc_fence_after();
-      const uint32_t slot = lane_addr + kMxSfBase + uint32_t(32 * s);
+      const uint32_t slot = lane_addr + C::kSfBase + uint32_t(32 * s);
       mx_tmem_st_x4(slot, sa[0], sa[1], sa[2], sa[3]);  // column j: rows 32j + lane
       mx_tmem_st_x8(slot + 16, sb);                      // column j: output columns 32j .. 32j + 31
       mx_tmem_st_wait();
@@ -385,18 +397,18 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; item < items && (kSplitK || ok); item += gridDim.x, ++tile_it) {
       const MxItem w = mx_item(p, item);
-      const int b = tile_it & 1;
+      const int b = tile_it % NB;
       const int row0 = w.tm * kMxBM + 32 * q;
-      const int col_base = w.tn * kMxBN + h * (kMxBN / 2);
-      if (ok && !__all_sync(0xffffffffu, mx_wait(tfull_bar(b), (tile_it >> 1) & 1, abort_flag, lim))) ok = false;
+      const int col_base = w.tn * BN + h * (BN / 2);
+      if (ok && !__all_sync(0xffffffffu, mx_wait(tfull_bar(b), (tile_it / NB) & 1, abort_flag, lim))) ok = false;
       if (ok) {
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < kMxBN / 64; ++c) {  // 3 chunks of 32 columns
+        for (int c = 0; c < BN / 64; ++c) {  // chunks of 32 columns
           uint32_t r[32];
-          tmem_ld_32x32b_x32(lane_addr + uint32_t(b * kMxBN + h * (kMxBN / 2) + 32 * c), r);
+          tmem_ld_32x32b_x32(lane_addr + uint32_t(b * BN + h * (BN / 2) + 32 * c), r);
           tmem_ld_wait();
-          if (c == kMxBN / 64 - 1) {
+          if (c == BN / 64 - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(b));
@@ -428,10 +440,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
           } else {
             const int row = row0 + lane;
             if (row < p.M) {
-              float* part_item = p.part + int64_t(item) * kMxBM * kMxBN;
+              float* part_item = p.part + int64_t(item) * kMxBM * BN;
 #pragma unroll
               for (int j = 0; j < 32; j += 4)
-                __stcg(reinterpret_cast<float4*>(splitk_quad(part_item, kMxBM, 32 * q + lane, h * (kMxBN / 2) + 32 * c + j)),
+                __stcg(reinterpret_cast<float4*>(splitk_quad(part_item, kMxBM, 32 * q + lane, h * (BN / 2) + 32 * c + j)),
                        make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
                                    __uint_as_float(r[j + 3])));
             }
@@ -440,13 +452,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
       }
       if constexpr (kSplitK) {
         // publish this split and finish the tile (splitk.cuh): the partials in split order
-        const int trow0 = w.tm * kMxBM, tcol0 = w.tn * kMxBN;
+        const int trow0 = w.tm * kMxBM, tcol0 = w.tn * BN;
         SplitTile t;
-        t.part = p.part + int64_t(w.tile) * p.splits * kMxBM * kMxBN;
-        t.split_elems = kMxBM * kMxBN;
+        t.part = p.part + int64_t(w.tile) * p.splits * kMxBM * BN;
+        t.split_elems = kMxBM * BN;
         t.bm = kMxBM;
         t.rows = min(kMxBM, p.M - trow0);
-        t.qpr = min(kMxBN, p.N - tcol0) / 4;
+        t.qpr = min(BN, p.N - tcol0) / 4;
         __nv_bfloat16* out_t = p.out + (int64_t(w.bt) * p.M + trow0) * p.N + tcol0;
         auto store = [&](int r, int c, float4 s) {
           *reinterpret_cast<uint2*>(out_t + int64_t(r) * p.N + c) =
@@ -490,9 +502,20 @@ static bool make_map_3d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tile width: 192 (two accumulators, tiles overlap on a persistent grid), unless 192-wide
+// tiles would spill into a partial second wave that 256-wide tiles avoid (e.g. M = 768,
+// N = 5120: 162 tiles of 192 on 148 SMs, 120 of 256); then 256 with one accumulator.
+static int mx_bn(int64_t batch, int64_t M, int64_t N) {
+  const int64_t sms = device_sm_count();
+  const int64_t mt = batch * ((M + kMxBM - 1) / kMxBM);
+  const int64_t t192 = mt * ((N + 191) / 192), t256 = mt * ((N + 255) / 256);
+  return (t192 > sms && t256 <= sms) ? 256 : 192;
+}
+
 static int mx_splits(int64_t batch, int64_t M, int64_t N, int64_t K) {
   const int64_t kb = K / 128;
-  const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + kMxBN - 1) / kMxBN);
+  const int bn = mx_bn(batch, M, N);
+  const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + bn - 1) / bn);
   const int64_t sms = device_sm_count();
   // one wave (tiles x splits <= SMs), at most 8 splits (the finish loads every split of an
   // element at once), each split at least 2 K blocks
@@ -505,8 +528,9 @@ static int mx_splits(int64_t batch, int64_t M, int64_t N, int64_t K) {
 size_t mx_workspace_bytes(int64_t batch, int64_t M, int64_t N, int64_t K) {
   const int sp = mx_splits(batch, M, N, K);
   if (sp == 1) return 0;
-  const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + kMxBN - 1) / kMxBN);
-  return kCounterBytes + size_t(tiles) * sp * kMxBM * kMxBN * sizeof(float);
+  const int bn = mx_bn(batch, M, N);
+  const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + bn - 1) / bn);
+  return kCounterBytes + size_t(tiles) * sp * kMxBM * bn * sizeof(float);
 }
 
 int launch_gemm_mx32(const void* A, const uint8_t* a_e, const void* W, const uint8_t* w_e, void* out, int64_t batch,
@@ -522,7 +546,8 @@ int launch_gemm_mx32(const void* A, const uint8_t* a_e, const void* W, const uin
   p.NB32 = int((N + 31) / 32);
   p.batch = int(batch);
   p.m_tiles = int((M + kMxBM - 1) / kMxBM);
-  p.n_tiles = int((N + kMxBN - 1) / kMxBN);
+  const int bn = mx_bn(batch, M, N);
+  p.n_tiles = int((N + bn - 1) / bn);
   p.splits = mx_splits(batch, M, N, K);
   p.wait_ns = wait_ns;
   if (p.splits > 1) {
@@ -532,19 +557,20 @@ int launch_gemm_mx32(const void* A, const uint8_t* a_e, const void* W, const uin
   }
   CUtensorMap ma, mb, mo;
   if (!make_map_3d(&ma, A, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, batch, 128, kMxBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_3d(&mb, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, batch, 128, kMxBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_3d(&mb, W, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, batch, 128, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_3d(&mo, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, batch, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return int(cudaErrorInvalidValue);
   const int items = p.batch * p.m_tiles * p.n_tiles * p.splits;
   const int grid = std::min(items, device_sm_count());
-  if (p.splits > 1) {
-    if (const int e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_mx_kernel<true>), int(kMxSmemBytes)))
-      return e;
-    return launch_kernel(gemm_mx_kernel<true>, dim3(grid), dim3(kMxThreads), kMxSmemBytes, stream, ma, mb, mo, p);
-  }
-  if (const int e = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_mx_kernel<false>), int(kMxSmemBytes)))
-    return e;
-  return launch_kernel(gemm_mx_kernel<false>, dim3(grid), dim3(kMxThreads), kMxSmemBytes, stream, ma, mb, mo, p);
+  auto go = [&](auto kernel, size_t smem) {
+    if (const int e = set_max_dynamic_smem(reinterpret_cast<const void*>(kernel), int(smem))) return e;
+    return launch_kernel(kernel, dim3(grid), dim3(kMxThreads), smem, stream, ma, mb, mo, p);
+  };
+  if (bn == 256)
+    return p.splits > 1 ? go(gemm_mx_kernel<true, 256>, MxCfg<256>::kSmemBytes)
+                        : go(gemm_mx_kernel<false, 256>, MxCfg<256>::kSmemBytes);
+  return p.splits > 1 ? go(gemm_mx_kernel<true, 192>, MxCfg<192>::kSmemBytes)
+                      : go(gemm_mx_kernel<false, 192>, MxCfg<192>::kSmemBytes);
 }
 
 }  // namespace fp8bs
