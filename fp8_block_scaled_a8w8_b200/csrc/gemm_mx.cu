@@ -119,7 +119,8 @@ __device__ __forceinline__ uint32_t mx_timer() {
   asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
   return t;
 }
-// Bounded wait (sleeping in try_wait between checks of the abort flag and the clock).
+// Bounded wait (sleeping in try_wait, at most 1 us at a time, between checks of the abort
+// flag and the clock; a longer suspend hint delays some resumes, as in the a8w8 kernels).
 __device__ __forceinline__ bool mx_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint32_t t0 = mx_timer();
@@ -130,7 +131,7 @@ __device__ __forceinline__ bool mx_wait(uint32_t bar, uint32_t parity, volatile 
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(50000u)
+        : "r"(bar), "r"(parity), "r"(1000u)
         : "memory");
     if (ok) return true;
     if (*abort) return false;
