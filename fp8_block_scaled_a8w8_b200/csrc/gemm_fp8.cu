@@ -20,9 +20,11 @@
 // buffers fill the 512 TMEM columns; with BN = 128 there are four.
 //
 // Split K (for shapes whose tiles leave SMs idle): a work item is (tile, K range); each
-// split stores its float32 partial tile and the last split to arrive (gpu-scope acq_rel
-// counter) sums the partials in split order -- a fixed order, so results are
-// bit-reproducible -- and rounds once to bf16.
+// split stores its float32 partial tile and the tile is finished by the shared split-K
+// finish (splitk.cuh): with one item per CTA every split sums its own share of the tile
+// once all have published, otherwise the last split to arrive sums it. The partials are
+// added in split order -- a fixed order, so results are bit-reproducible -- and rounded
+// once to bf16.
 //
 // Every wait is bounded by a limit passed in the kernel parameters (1 s by default); a
 // wait that gives up raises the CTA's abort flag and the device status word, the roles
