@@ -97,3 +97,30 @@ def test_weight_streaming_workspace(M, N, K):
     assert fb.workspace_bytes(fb.OP_A8W8_BLOCKSCALE, M, N, K) == max(own8, tma)
     own16 = KCOUNTER + 2 * ctas(nblk * (K // 64)) * 32 * 128 * 4
     assert fb.workspace_bytes(fb.OP_BF16, M, N, K) == own16
+
+
+def _mx_bn(batch, M, N):
+    mt = batch * math.ceil(M / 128)
+    t192, t256 = mt * math.ceil(N / 192), mt * math.ceil(N / 256)
+    return 256 if (t192 > SMS and t256 <= SMS) else 192
+
+
+@pytest.mark.parametrize("batch,M,N,K", [(1, 48, 1792, 5120), (1, 768, 1792, 5120), (1, 48, 4608, 5120),
+                                         (1, 768, 4608, 5120), (1, 768, 5120, 2304), (1, 768, 5120, 8192),
+                                         (1, 48, 32768, 1280), (8, 16, 1024, 4096), (8, 64, 1024, 4096),
+                                         (1, 1, 192, 128), (1, 40, 256, 256)])
+def test_mx32_tiles_and_splits(batch, M, N, K):
+    """MX32: 192-wide tiles, or 256-wide ones (one accumulator) when 192-wide tiles would
+    spill into a partial second wave that 256-wide tiles avoid; K is split only when the
+    tiles leave half the SMs idle, into as many splits as keep one wave, at most 8, each at
+    least 2 K blocks (workspace = counters + one fp32 partial tile per split)."""
+    kb = K // 128
+    bn = _mx_bn(batch, M, N)
+    tiles = batch * math.ceil(M / 128) * math.ceil(N / bn)
+    sp = 1 if 2 * tiles >= SMS else max(1, min(SMS // tiles, kb // 2, 8, kb))
+    want = 0 if sp == 1 else KCOUNTER + tiles * sp * 128 * bn * 4
+    assert fb.mx32_workspace_bytes(batch, M, N, K) == want
+    if (batch, M, N, K) == (1, 768, 5120, 8192):
+        assert bn == 256 and sp == 1  # 162 tiles of 192 against 120 of 256 on 148 SMs
+    if (batch, M, N, K) == (1, 48, 1792, 5120):
+        assert bn == 192 and sp == 8
