@@ -503,33 +503,45 @@ static bool make_map_3d(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tile width: 192 (two accumulators, tiles overlap on a persistent grid), unless 192-wide
-// tiles would spill into a partial second wave that 256-wide tiles avoid (e.g. M = 768,
-// N = 5120: 162 tiles of 192 on 148 SMs, 120 of 256); then 256 with one accumulator.
-static int mx_bn(int64_t batch, int64_t M, int64_t N) {
+// K splits of a one-wave split launch: as many as keep tiles x splits within the SMs, at
+// most 8 (the finish loads every split of an element at once), each at least 2 K blocks.
+static int64_t mx_auto_splits(int64_t tiles, int64_t kb) {
   const int64_t sms = device_sm_count();
-  const int64_t mt = batch * ((M + kMxBM - 1) / kMxBM);
-  const int64_t t192 = mt * ((N + 191) / 192), t256 = mt * ((N + 255) / 256);
-  return (t192 > sms && t256 <= sms) ? 256 : 192;
-}
-
-static int mx_splits(int64_t batch, int64_t M, int64_t N, int64_t K) {
-  const int64_t kb = K / 128;
-  const int bn = mx_bn(batch, M, N);
-  const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + bn - 1) / bn);
-  const int64_t sms = device_sm_count();
-  // one wave (tiles x splits <= SMs), at most 8 splits (the finish loads every split of an
-  // element at once), each split at least 2 K blocks
   int64_t sp = 2 * tiles >= sms ? 1 : std::min<int64_t>({sms / tiles, kb / 2, 8});
   sp = std::max<int64_t>(1, std::min(sp, kb));
   if (sp > 1 && tiles > kMaxCounters) sp = 1;
-  return int(sp);
+  return sp;
+}
+
+// Tile width: 192 (two accumulators, tiles overlap on a persistent grid), unless 192-wide
+// tiles would spill into a partial second wave that 256-wide tiles avoid (e.g. M = 768,
+// N = 5120: 162 tiles of 192 on 148 SMs, 120 of 256); then 256 with one accumulator. A
+// single GEMM whose 192-wide tiles split K also takes 256-wide tiles when their split
+// leaves each CTA fewer K stages, a 256-wide stage counted as 1.15 of a 192-wide one
+// (measured on a B200: M = 768, N = 1792, K = 5120 20.3 -> 18.6 us; M = 48, N = 4608 12.4
+// -> 11.9 us; batched calls ran 2-4 % slower, so they keep 192).
+static int mx_bn(int64_t batch, int64_t M, int64_t N, int64_t K) {
+  const int64_t sms = device_sm_count();
+  const int64_t mt = batch * ((M + kMxBM - 1) / kMxBM);
+  const int64_t t192 = mt * ((N + 191) / 192), t256 = mt * ((N + 255) / 256);
+  if (t192 > sms && t256 <= sms) return 256;
+  if (batch == 1 && 2 * t192 < sms) {
+    const int64_t kb = K / 128;
+    const int64_t s192 = mx_auto_splits(t192, kb), s256 = mx_auto_splits(t256, kb);
+    if (115 * ((kb + s256 - 1) / s256) < 100 * ((kb + s192 - 1) / s192)) return 256;
+  }
+  return 192;
+}
+
+static int mx_splits(int64_t batch, int64_t M, int64_t N, int64_t K) {
+  const int bn = mx_bn(batch, M, N, K);
+  return int(mx_auto_splits(batch * ((M + kMxBM - 1) / kMxBM) * ((N + bn - 1) / bn), K / 128));
 }
 
 size_t mx_workspace_bytes(int64_t batch, int64_t M, int64_t N, int64_t K) {
   const int sp = mx_splits(batch, M, N, K);
   if (sp == 1) return 0;
-  const int bn = mx_bn(batch, M, N);
+  const int bn = mx_bn(batch, M, N, K);
   const int64_t tiles = batch * ((M + kMxBM - 1) / kMxBM) * ((N + bn - 1) / bn);
   return kCounterBytes + size_t(tiles) * sp * kMxBM * bn * sizeof(float);
 }
@@ -547,7 +559,7 @@ int launch_gemm_mx32(const void* A, const uint8_t* a_e, const void* W, const uin
   p.NB32 = int((N + 31) / 32);
   p.batch = int(batch);
   p.m_tiles = int((M + kMxBM - 1) / kMxBM);
-  const int bn = mx_bn(batch, M, N);
+  const int bn = mx_bn(batch, M, N, K);
   p.n_tiles = int((N + bn - 1) / bn);
   p.splits = mx_splits(batch, M, N, K);
   p.wait_ns = wait_ns;

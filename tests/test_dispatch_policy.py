@@ -99,10 +99,20 @@ def test_weight_streaming_workspace(M, N, K):
     assert fb.workspace_bytes(fb.OP_BF16, M, N, K) == own16
 
 
-def _mx_bn(batch, M, N):
+def _mx_split(tiles, kb):
+    return 1 if 2 * tiles >= SMS else max(1, min(SMS // tiles, kb // 2, 8, kb))
+
+
+def _mx_bn(batch, M, N, K):
     mt = batch * math.ceil(M / 128)
     t192, t256 = mt * math.ceil(N / 192), mt * math.ceil(N / 256)
-    return 256 if (t192 > SMS and t256 <= SMS) else 192
+    if t192 > SMS and t256 <= SMS:
+        return 256
+    if batch == 1 and 2 * t192 < SMS:  # fewer K stages per CTA at 1.15 the cost per stage
+        kb = K // 128
+        if 115 * math.ceil(kb / _mx_split(t256, kb)) < 100 * math.ceil(kb / _mx_split(t192, kb)):
+            return 256
+    return 192
 
 
 @pytest.mark.parametrize("batch,M,N,K", [(1, 48, 1792, 5120), (1, 768, 1792, 5120), (1, 48, 4608, 5120),
@@ -111,16 +121,22 @@ def _mx_bn(batch, M, N):
                                          (1, 1, 192, 128), (1, 40, 256, 256)])
 def test_mx32_tiles_and_splits(batch, M, N, K):
     """MX32: 192-wide tiles, or 256-wide ones (one accumulator) when 192-wide tiles would
-    spill into a partial second wave that 256-wide tiles avoid; K is split only when the
-    tiles leave half the SMs idle, into as many splits as keep one wave, at most 8, each at
-    least 2 K blocks (workspace = counters + one fp32 partial tile per split)."""
+    spill into a partial second wave that 256-wide tiles avoid, or, for a single GEMM that
+    splits K, when 256-wide tiles leave each CTA fewer K stages (a stage counted 1.15 times);
+    K is split only when the tiles leave half the SMs idle, into as many splits as keep one
+    wave, at most 8, each at least 2 K blocks (workspace = counters + one fp32 partial tile
+    per split)."""
     kb = K // 128
-    bn = _mx_bn(batch, M, N)
+    bn = _mx_bn(batch, M, N, K)
     tiles = batch * math.ceil(M / 128) * math.ceil(N / bn)
-    sp = 1 if 2 * tiles >= SMS else max(1, min(SMS // tiles, kb // 2, 8, kb))
+    sp = _mx_split(tiles, kb)
     want = 0 if sp == 1 else KCOUNTER + tiles * sp * 128 * bn * 4
     assert fb.mx32_workspace_bytes(batch, M, N, K) == want
     if (batch, M, N, K) == (1, 768, 5120, 8192):
         assert bn == 256 and sp == 1  # 162 tiles of 192 against 120 of 256 on 148 SMs
     if (batch, M, N, K) == (1, 48, 1792, 5120):
         assert bn == 192 and sp == 8
+    if (batch, M, N, K) == (1, 768, 1792, 5120):
+        assert bn == 256 and sp == 3  # 42 tiles x 3 splits: 14 K blocks a CTA against 20
+    if batch == 8:
+        assert bn == 192

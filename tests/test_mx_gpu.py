@@ -66,7 +66,9 @@ def _run(A, ae, W, we, ws=None):
 @pytest.mark.parametrize("M,N,K", [(1, 192, 128), (16, 256, 512), (48, 1792, 5120), (130, 2320, 384),
                                    (300, 4608, 512), (257, 1024, 1280), (600, 5120, 640),
                                    # 256-wide tiles (192-wide ones would need a partial second wave)
-                                   (768, 5120, 512), (800, 4800, 384)])
+                                   (768, 5120, 512), (800, 4800, 384),
+                                   # 256-wide tiles with K split three ways (192-wide: two ways)
+                                   (768, 1792, 2048)])
 def test_gemm_mx32_parity(M, N, K):
     case = _raw(M, N, K, M + N + K)
     check_mx32(_run(*case), *case)
