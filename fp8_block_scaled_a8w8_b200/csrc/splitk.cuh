@@ -21,6 +21,13 @@
 // Either way all of an element's split loads are issued before its first add, and the
 // elements are spread over every thread of the epilogue, so the finish costs one L2 round
 // trip per batch of elements rather than one per split and column chunk.
+//
+// Ordering: the epilogue threads' partial stores (st.global.cg) precede a barrier of the
+// epilogue group, after which one thread's release add publishes them at gpu scope (the
+// barrier orders the other threads' stores before that release); a thread whose acquire
+// load observes every arrival, followed by a barrier of the group, orders all the group's
+// partial loads (ld.global.cg) after the other CTAs' stores. Plain weak polling would not
+// do: it is not guaranteed to observe a store made on the other die's L2 partition.
 #pragma once
 
 #include <cuda_runtime.h>
